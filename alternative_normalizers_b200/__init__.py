@@ -1,0 +1,25 @@
+"""B200-native fused attention with selectable row normalizers.
+
+``O = N(scale * Q K^T + mask) V`` with N one of softmax, softmax1, sparsemax
+and 1.5-entmax, computed by the CUDA kernels of ``libnattn.so`` (sm_100a).
+The Python layer only allocates with PyTorch and marshals arguments; build the
+library with ``python -m alternative_normalizers_b200.build``.
+"""
+
+from .binding import (  # noqa: F401
+    NattnArgs,
+    NattnError,
+    attention,
+    build_args,
+    lib,
+    nattn_fwd,
+    nattn_fwd_ex,
+    nattn_get_device_status,
+    nattn_strerror,
+    nattn_version,
+    nattn_workspace_size,
+    paged_attention,
+)
+from .workloads import NORMALIZER_IDS, WORKLOADS, Workload  # noqa: F401
+
+__version__ = "0.1.0"

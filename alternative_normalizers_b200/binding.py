@@ -1,0 +1,218 @@
+"""ctypes binding of libnattn (include/nattn.h).
+
+Argument marshalling only: every step of the attention forward runs in the
+library's CUDA kernels.  PyTorch supplies device memory and the current
+stream; nothing here computes attention.  If the shared library is missing
+the first call raises, there is no other implementation to fall back on.
+"""
+
+import ctypes
+import os
+
+from .workloads import NORMALIZER_IDS
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libnattn.so")
+
+NATTN_OK = 0
+ERRORS = {
+    -1: "NATTN_EINVAL", -2: "NATTN_EUNSUPPORTED", -3: "NATTN_ETOOLARGE",
+    -4: "NATTN_EWORKSPACE", -5: "NATTN_ECUDA", -6: "NATTN_ETIMEOUT",
+    -7: "NATTN_EBOUNDS", -8: "NATTN_EALIGN",
+}
+
+
+class NattnArgs(ctypes.Structure):
+    """Mirror of ``nattn_args``."""
+
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("out", ctypes.c_void_p), ("row_stat", ctypes.c_void_p),
+        ("weights", ctypes.c_void_p),
+        ("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+        ("Tq", ctypes.c_int), ("Tk", ctypes.c_int), ("d", ctypes.c_int),
+        ("dv", ctypes.c_int),
+        ("scale", ctypes.c_float), ("normalizer", ctypes.c_int),
+        ("causal", ctypes.c_int), ("window", ctypes.c_int),
+        ("softcap", ctypes.c_float),
+        ("block_table", ctypes.c_void_p), ("seqlens", ctypes.c_void_p),
+        ("page_size", ctypes.c_int), ("block_table_stride", ctypes.c_int),
+        ("num_pages", ctypes.c_int),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("stream", ctypes.c_void_p),
+    ]
+
+
+class NattnError(RuntimeError):
+    def __init__(self, code, where):
+        self.code = code
+        super().__init__(f"{where}: {ERRORS.get(code, code)} "
+                         f"({nattn_strerror(code)})")
+
+
+_lib = None
+
+
+def lib():
+    """Load libnattn.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"libnattn.so not found at {LIB_PATH}; build it with "
+                "`python -m alternative_normalizers_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER(NattnArgs)
+        L.nattn_fwd_ex.argtypes = [P]
+        L.nattn_fwd_ex.restype = ctypes.c_int
+        L.nattn_workspace_size.argtypes = [P]
+        L.nattn_workspace_size.restype = ctypes.c_size_t
+        L.nattn_fwd.argtypes = (
+            [ctypes.c_void_p] * 4 + [ctypes.c_void_p]
+            + [ctypes.c_int] * 7 + [ctypes.c_float, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_int, ctypes.c_float]
+            + [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p])
+        L.nattn_fwd.restype = ctypes.c_int
+        L.nattn_get_device_status.argtypes = [ctypes.c_void_p]
+        L.nattn_get_device_status.restype = ctypes.c_int
+        L.nattn_strerror.argtypes = [ctypes.c_int]
+        L.nattn_strerror.restype = ctypes.c_char_p
+        L.nattn_version.argtypes = []
+        L.nattn_version.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+# --------------------------------------------------------------------------
+# The C entry points under their own names
+# --------------------------------------------------------------------------
+
+def nattn_fwd(q, k, v, out, row_stat, B, Hq, Hkv, Tq, Tk, d, dv, scale,
+              normalizer, causal, window, softcap, block_table, seqlens,
+              stream):
+    """``nattn_fwd`` with raw device pointers (ints) and sizes."""
+    return lib().nattn_fwd(q, k, v, out, row_stat, B, Hq, Hkv, Tq, Tk, d, dv,
+                           scale, normalizer, causal, window, softcap,
+                           block_table, seqlens, stream)
+
+
+def nattn_fwd_ex(args: NattnArgs):
+    return lib().nattn_fwd_ex(ctypes.byref(args))
+
+
+def nattn_workspace_size(args: NattnArgs):
+    return lib().nattn_workspace_size(ctypes.byref(args))
+
+
+def nattn_get_device_status(stream=None):
+    return lib().nattn_get_device_status(stream)
+
+
+def nattn_strerror(code):
+    return lib().nattn_strerror(code).decode()
+
+
+def nattn_version():
+    return lib().nattn_version()
+
+
+# --------------------------------------------------------------------------
+# torch-tensor front ends (allocation + marshalling)
+# --------------------------------------------------------------------------
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _norm_id(normalizer):
+    if isinstance(normalizer, str):
+        return NORMALIZER_IDS[normalizer]
+    return int(normalizer)
+
+
+def build_args(q, k, v, out, row_stat=None, weights=None, *, normalizer,
+               causal=False, window=0, softcap=0.0, scale=None,
+               block_table=None, seqlens=None, page_size=0, max_seqlen=None,
+               stream=None):
+    """Fill an ``NattnArgs`` from torch tensors (no device work)."""
+    import torch
+    B, Hq, Tq, d = q.shape
+    a = NattnArgs()
+    a.q, a.k, a.v, a.out = _ptr(q), _ptr(k), _ptr(v), _ptr(out)
+    a.row_stat, a.weights = _ptr(row_stat), _ptr(weights)
+    a.B, a.Hq, a.Tq, a.d = B, Hq, Tq, d
+    a.Hkv = k.shape[1]
+    a.dv = v.shape[3]
+    a.scale = (1.0 / d ** 0.5) if scale is None else scale
+    a.normalizer = _norm_id(normalizer)
+    a.causal, a.window, a.softcap = int(bool(causal)), int(window), float(softcap)
+    if block_table is not None:
+        a.block_table, a.seqlens = _ptr(block_table), _ptr(seqlens)
+        a.page_size = page_size or k.shape[2]
+        a.block_table_stride = block_table.shape[1]
+        a.num_pages = k.shape[0]
+        a.Tk = int(max_seqlen)
+    else:
+        a.Tk = k.shape[2]
+    if stream is None and q.is_cuda:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    a.stream = stream
+    return a
+
+
+def _run(a, workspace_holder):
+    import torch
+    need = nattn_workspace_size(a)
+    ws = None
+    if need:
+        ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+        a.workspace, a.workspace_bytes = ws.data_ptr(), need
+    workspace_holder.append(ws)
+    rc = nattn_fwd_ex(a)
+    if rc != NATTN_OK:
+        raise NattnError(rc, "nattn_fwd_ex")
+
+
+def attention(q, k, v, normalizer="softmax", causal=False, window=0,
+              softcap=0.0, scale=None, want_weights=False, out=None,
+              row_stat=None):
+    """Dense attention forward.  q [B,Hq,Tq,d], k [B,Hkv,Tk,d], v
+    [B,Hkv,Tk,dv] (bf16, CUDA, contiguous).  Returns (out, row_stat,
+    weights|None)."""
+    import torch
+    B, Hq, Tq, _ = q.shape
+    Tk, dv = k.shape[2], v.shape[3]
+    out = torch.empty(B, Hq, Tq, dv, dtype=torch.bfloat16, device=q.device) \
+        if out is None else out
+    row_stat = torch.empty(B, Hq, Tq, dtype=torch.float32, device=q.device) \
+        if row_stat is None else row_stat
+    weights = torch.empty(B, Hq, Tq, Tk, dtype=torch.float32,
+                          device=q.device) if want_weights else None
+    a = build_args(q, k, v, out, row_stat, weights, normalizer=normalizer,
+                   causal=causal, window=window, softcap=softcap, scale=scale)
+    keep = []
+    _run(a, keep)
+    return out, row_stat, weights
+
+
+def paged_attention(q, k_pool, v_pool, block_table, seqlens, max_seqlen,
+                    normalizer="softmax", causal=True, window=0, softcap=0.0,
+                    scale=None, out=None, row_stat=None):
+    """Attention of q [B,Hq,Tq,d] over a paged cache: k_pool/v_pool
+    [num_pages, Hkv, page, d], block_table int32 [B, max_pages], seqlens
+    int32 [B] (each <= max_seqlen)."""
+    import torch
+    B, Hq, Tq, _ = q.shape
+    dv = v_pool.shape[3]
+    out = torch.empty(B, Hq, Tq, dv, dtype=torch.bfloat16, device=q.device) \
+        if out is None else out
+    row_stat = torch.empty(B, Hq, Tq, dtype=torch.float32, device=q.device) \
+        if row_stat is None else row_stat
+    a = build_args(q, k_pool, v_pool, out, row_stat, None,
+                   normalizer=normalizer, causal=causal, window=window,
+                   softcap=softcap, scale=scale, block_table=block_table,
+                   seqlens=seqlens, page_size=k_pool.shape[2],
+                   max_seqlen=max_seqlen)
+    keep = []
+    _run(a, keep)
+    return out, row_stat

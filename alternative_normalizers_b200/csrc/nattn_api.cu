@@ -1,0 +1,495 @@
+// libnattn host side: argument validation, scratch layout, TMA descriptors and
+// kernel dispatch behind the C ABI declared in include/nattn.h.
+//
+// Dispatch (no fallback between backends; each request has one path):
+//   dense weights requested              -> row-wise kernel
+//   paged KV, supported shape            -> split-KV decode kernels
+//   dense, head dims 64/128/256 (d == dv)-> tcgen05 prefill kernels
+//   anything else that validates         -> row-wise kernel
+#include <math.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "prefill_tc.cuh"
+#include "problem.cuh"
+#include "rowwise.cuh"
+
+using namespace nattn;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr int kMaxDevices = 64;
+constexpr int kRowSmemCap = 48 * 1024;  // scores kept in shared memory per row
+constexpr long long kMaxWeights = 1ll << 26;
+
+// ---------------------------------------------------------------------------
+// TMA descriptor encoding through the driver entry point (no -lcuda needed)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                         cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// bf16 tensor viewed as [outer][rows][inner] with a (64 x box_rows) box and
+// the 128-byte swizzle.  Rows past `rows` read as zero.
+bool make_map_3d(CUtensorMap* m, const void* base, int inner, int rows, long long outer,
+                 int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)outer};
+  cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)inner * 2 * rows};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_2d(CUtensorMap* m, const void* base, int inner, long long rows, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)inner * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Per-device one-time kernel attribute set-up (dynamic shared memory opt-in).
+template <class K>
+cudaError_t allow_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// ---------------------------------------------------------------------------
+// Path selection and scratch sizing
+// ---------------------------------------------------------------------------
+enum Path { PATH_NONE, PATH_ROWWISE, PATH_TC, PATH_DECODE };
+
+struct Plan {
+  Path path = PATH_NONE;
+  bool sparse = false;
+  // decode
+  int R = 0, nsplit = 0, pps = 0;
+  // scratch offsets (bytes)
+  size_t off_tau = 0, off_ovfc = 0, off_ovfr = 0, off_slots = 0;
+  size_t off_opart = 0, off_ml = 0, off_scores = 0;
+  size_t total = 0;
+  int row_grid = 0, row_cap = 0;
+  bool row_slots = false;
+};
+
+bool is_paged(const nattn_args* a) { return a->block_table != nullptr; }
+
+int validate(const nattn_args* a) {
+  if (a == nullptr) return NATTN_EINVAL;
+  if (a->B < 0 || a->Hq < 0 || a->Tq < 0 || a->Tk < 0) return NATTN_EINVAL;
+  if (a->B == 0 || a->Hq == 0 || a->Tq == 0) return NATTN_OK;  // nothing to compute
+  if (a->Hkv < 1 || a->Hq % a->Hkv != 0) return NATTN_EINVAL;
+  if (a->d < 8 || a->d > 256 || a->d % 8 || a->dv < 8 || a->dv > 256 || a->dv % 8)
+    return NATTN_EUNSUPPORTED;
+  if (!(a->scale == a->scale) || isinf(a->scale)) return NATTN_EINVAL;
+  if (!(a->softcap >= 0.f) || isinf(a->softcap)) return NATTN_EINVAL;
+  if (a->window < 0) return NATTN_EINVAL;
+  if (a->normalizer < 0 || a->normalizer > 3) return NATTN_EINVAL;
+  if (a->causal != 0 && a->causal != 1) return NATTN_EINVAL;
+  if (!a->q || !a->k || !a->v || !a->out) return NATTN_EINVAL;
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out))
+    return NATTN_EALIGN;
+  if ((a->row_stat && (reinterpret_cast<uintptr_t>(a->row_stat) & 3)) ||
+      (a->weights && (reinterpret_cast<uintptr_t>(a->weights) & 3)))
+    return NATTN_EALIGN;
+  const long long rows = (long long)a->B * a->Hq * a->Tq;
+  if (rows >= (1ll << 31) || rows * (long long)(a->d > a->dv ? a->d : a->dv) >= (1ll << 40))
+    return NATTN_ETOOLARGE;
+  if (is_paged(a)) {
+    if (!a->seqlens || a->page_size < 1 || a->block_table_stride < 1 || a->num_pages < 1 ||
+        a->Tk < 1)
+      return NATTN_EINVAL;
+    if (a->weights) return NATTN_EUNSUPPORTED;
+    if ((long long)a->num_pages * a->Hkv * a->page_size >= (1ll << 31))
+      return NATTN_ETOOLARGE;
+  } else {
+    if ((long long)a->B * a->Hkv * a->Tk >= (1ll << 31)) return NATTN_ETOOLARGE;
+    if (a->weights && rows * (long long)a->Tk > kMaxWeights) return NATTN_ETOOLARGE;
+  }
+  return NATTN_OK;
+}
+
+int decode_pps() {
+  const char* e = getenv("NATTN_DECODE_PPS");
+  int v = e ? atoi(e) : 0;
+  return (v >= 1 && v <= 256) ? v : 32;
+}
+
+Plan make_plan(const nattn_args* a) {
+  Plan pl;
+  const bool sparse = a->normalizer == NATTN_SPARSEMAX || a->normalizer == NATTN_ENTMAX15;
+  pl.sparse = sparse;
+  const size_t rows = (size_t)a->B * a->Hq * a->Tq;
+  const int group = a->Hq / a->Hkv;
+  const bool tc_dims = a->d == a->dv && (a->d == 64 || a->d == 128 || a->d == 256);
+  if (is_paged(a)) {
+    const bool ps_ok = a->page_size == 32 || a->page_size == 64;
+    if (tc_dims && ps_ok && group * a->Tq <= 16) {
+      pl.path = PATH_DECODE;
+      pl.R = group * a->Tq;
+      const int maxp = (a->Tk + a->page_size - 1) / a->page_size;
+      pl.pps = decode_pps();
+      if (pl.pps > maxp) pl.pps = maxp;
+      pl.nsplit = (maxp + pl.pps - 1) / pl.pps;
+      const size_t parts = (size_t)a->B * a->Hkv * pl.nsplit * pl.R;
+      size_t off = 0;
+      pl.off_opart = off;
+      off = up256(off + parts * a->dv * 4);
+      pl.off_ml = off;
+      off = up256(off + parts * 2 * 4);
+      if (sparse) {
+        pl.off_scores = off;
+        off = up256(off + rows * (size_t)a->Tk * 4);
+        pl.off_tau = off;
+        off = up256(off + rows * 4);
+      }
+      pl.total = off;
+      return pl;
+    }
+  } else if (!a->weights && tc_dims && a->Tk >= 1) {
+    pl.path = PATH_TC;
+    if (sparse) {
+      size_t off = 0;
+      pl.off_tau = off;
+      off = up256(off + rows * 4);
+      pl.off_ovfc = off;
+      off = up256(off + 4);
+      pl.off_ovfr = off;
+      off = up256(off + rows * 4);
+      pl.row_grid = 2 * 148;
+      pl.row_cap = a->Tk < kRowSmemCap ? (a->Tk < 256 ? 256 : a->Tk) : kRowSmemCap;
+      if (a->Tk > kRowSmemCap) {
+        pl.row_slots = true;
+        pl.off_slots = off;
+        off = up256(off + (size_t)pl.row_grid * a->Tk * 4);
+      }
+      pl.total = off;
+    }
+    return pl;
+  }
+  // row-wise
+  pl.path = PATH_ROWWISE;
+  pl.row_grid = (int)(rows < 148 * 16 ? rows : 148 * 16);
+  if (pl.row_grid < 1) pl.row_grid = 1;
+  const int tk = a->Tk;
+  pl.row_cap = tk < kRowSmemCap ? (tk < 256 ? 256 : tk) : kRowSmemCap;
+  if (tk > kRowSmemCap) {
+    pl.row_slots = true;
+    pl.off_slots = 0;
+    pl.total = up256((size_t)pl.row_grid * tk * 4);
+  }
+  return pl;
+}
+
+Problem to_problem(const nattn_args* a) {
+  Problem P;
+  P.q = static_cast<const bf16*>(a->q);
+  P.k = static_cast<const bf16*>(a->k);
+  P.v = static_cast<const bf16*>(a->v);
+  P.out = static_cast<bf16*>(a->out);
+  P.row_stat = a->row_stat;
+  P.weights = a->weights;
+  P.B = a->B;
+  P.Hq = a->Hq;
+  P.Hkv = a->Hkv;
+  P.Tq = a->Tq;
+  P.Tk = a->Tk;
+  P.d = a->d;
+  P.dv = a->dv;
+  P.scale = a->scale;
+  P.norm = a->normalizer;
+  P.causal = a->causal;
+  P.window = a->window;
+  P.softcap = a->softcap;
+  P.block_table = a->block_table;
+  P.seqlens = a->seqlens;
+  P.page_size = a->page_size;
+  P.bt_stride = a->block_table_stride;
+  P.num_pages = a->num_pages;
+  return P;
+}
+
+int check_launch() {
+  return cudaGetLastError() == cudaSuccess ? NATTN_OK : NATTN_ECUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Launchers
+// ---------------------------------------------------------------------------
+int launch_rowwise(const Problem& P, const Plan& pl, const int* row_list,
+                   const int* row_count, int nrows, float* slots, int grid,
+                   cudaStream_t st) {
+  const int bytes = (256 + 64 + ROW_THREADS + pl.row_cap) * 4;
+  if (allow_smem(rowwise_kernel, bytes) != cudaSuccess) return NATTN_ECUDA;
+  rowwise_kernel<<<grid, ROW_THREADS, bytes, st>>>(P, row_list, row_count, nrows,
+                                                   pl.row_cap, slots);
+  return check_launch();
+}
+
+template <int D>
+int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws,
+              cudaStream_t st) {
+  constexpr int BN = (D == 256) ? 64 : 128;
+  constexpr int KST = 2, VST = 2;
+  CUtensorMap mq, mk, mv;
+  if (!make_map_3d(&mq, a->q, D, a->Tq, (long long)a->B * a->Hq, TC_BM) ||
+      !make_map_3d(&mk, a->k, D, a->Tk, (long long)a->B * a->Hkv, BN) ||
+      !make_map_3d(&mv, a->v, D, a->Tk, (long long)a->B * a->Hkv, BN))
+    return NATTN_ECUDA;
+  TcArgs A;
+  A.P = P;
+  const float log2e = 1.4426950408889634f;
+  const int ntq = (a->Tq + TC_BM - 1) / TC_BM;
+  const unsigned grid = (unsigned)((long long)a->B * a->Hq * ntq);
+  if (!pl.sparse) {
+    A.zscale = a->scale * log2e;
+    A.capscale = a->softcap * log2e;
+    A.tau = nullptr;
+    A.ovf_rows = nullptr;
+    A.ovf_count = nullptr;
+    using LY = TcLayout<D, D, BN, KST, VST, TC_ONLINE>;
+    auto k = prefill_tc_kernel<D, D, BN, KST, VST, TC_ONLINE>;
+    if (allow_smem(k, LY::ALLOC) != cudaSuccess) return NATTN_ECUDA;
+    k<<<grid, TC_THREADS, LY::ALLOC, st>>>(mq, mk, mv, A);
+    return check_launch();
+  }
+  const float us = (a->normalizer == NATTN_ENTMAX15) ? 0.5f : 1.0f;
+  A.zscale = a->scale * us;
+  A.capscale = a->softcap * us;
+  A.tau = reinterpret_cast<float*>(ws + pl.off_tau);
+  A.ovf_count = reinterpret_cast<int*>(ws + pl.off_ovfc);
+  A.ovf_rows = reinterpret_cast<int*>(ws + pl.off_ovfr);
+  if (cudaMemsetAsync(A.ovf_count, 0, sizeof(int), st) != cudaSuccess) return NATTN_ECUDA;
+  {
+    using LY = TcLayout<D, D, BN, 3, 1, TC_TAU>;
+    auto k = prefill_tc_kernel<D, D, BN, 3, 1, TC_TAU>;
+    if (allow_smem(k, LY::ALLOC) != cudaSuccess) return NATTN_ECUDA;
+    k<<<grid, TC_THREADS, LY::ALLOC, st>>>(mq, mk, mv, A);
+    if (check_launch() != NATTN_OK) return NATTN_ECUDA;
+  }
+  {
+    using LY = TcLayout<D, D, BN, KST, VST, TC_APPLY>;
+    auto k = prefill_tc_kernel<D, D, BN, KST, VST, TC_APPLY>;
+    if (allow_smem(k, LY::ALLOC) != cudaSuccess) return NATTN_ECUDA;
+    k<<<grid, TC_THREADS, LY::ALLOC, st>>>(mq, mk, mv, A);
+    if (check_launch() != NATTN_OK) return NATTN_ECUDA;
+  }
+  // rows whose candidate buffer overflowed: exact row-wise recomputation
+  float* slots = pl.row_slots ? reinterpret_cast<float*>(ws + pl.off_slots) : nullptr;
+  return launch_rowwise(P, pl, A.ovf_rows, A.ovf_count, 0, slots, pl.row_grid, st);
+}
+
+template <int D, int PS, int MODE>
+int launch_decode_mode(const nattn_args* a, const DecodeArgs& A, const CUtensorMap& mk,
+                       const CUtensorMap& mv, cudaStream_t st) {
+  using L1 = DecodeSmem<D, D, PS, 2, MODE>;
+  constexpr int NS = (L1::STAGE * 4 <= 128 * 1024) ? 4 : (L1::STAGE * 3 <= 200 * 1024 ? 3 : 2);
+  using L = DecodeSmem<D, D, PS, NS, MODE>;
+  const int bytes = L::BYTES_NOLIST + 2 * A.pps * 4 + 1024;
+  dim3 grid(A.nsplit, a->Hkv, a->B);
+  if (A.R <= 8) {
+    auto k = decode_split_kernel<D, D, PS, NS, 1, MODE>;
+    if (allow_smem(k, bytes) != cudaSuccess) return NATTN_ECUDA;
+    k<<<grid, DEC_THREADS, bytes, st>>>(mk, mv, A);
+  } else {
+    auto k = decode_split_kernel<D, D, PS, NS, 2, MODE>;
+    if (allow_smem(k, bytes) != cudaSuccess) return NATTN_ECUDA;
+    k<<<grid, DEC_THREADS, bytes, st>>>(mk, mv, A);
+  }
+  return check_launch();
+}
+
+template <int D, int PS>
+int launch_decode(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws,
+                  cudaStream_t st) {
+  CUtensorMap mk, mv;
+  const long long prow = (long long)a->num_pages * a->Hkv * PS;
+  if (!make_map_2d(&mk, a->k, D, prow, PS) || !make_map_2d(&mv, a->v, D, prow, PS))
+    return NATTN_ECUDA;
+  DecodeArgs A;
+  A.P = P;
+  A.R = pl.R;
+  A.nsplit = pl.nsplit;
+  A.pps = pl.pps;
+  A.opart = reinterpret_cast<float*>(ws + pl.off_opart);
+  A.ml = reinterpret_cast<float*>(ws + pl.off_ml);
+  A.scores = pl.sparse ? reinterpret_cast<float*>(ws + pl.off_scores) : nullptr;
+  A.tau = pl.sparse ? reinterpret_cast<float*>(ws + pl.off_tau) : nullptr;
+  const unsigned rows = (unsigned)((size_t)a->B * a->Hq * a->Tq);
+  if (!pl.sparse) {
+    A.zscale = a->scale * 1.4426950408889634f;
+    A.uscale = 1.f;
+    int rc = launch_decode_mode<D, PS, DEC_ONLINE>(a, A, mk, mv, st);
+    if (rc) return rc;
+    decode_combine_kernel<<<rows, 128, 0, st>>>(A, DEC_ONLINE);
+    return check_launch();
+  }
+  A.uscale = (a->normalizer == NATTN_ENTMAX15) ? 0.5f : 1.0f;
+  A.zscale = a->scale * A.uscale;
+  int rc = launch_decode_mode<D, PS, DEC_SCORES>(a, A, mk, mv, st);
+  if (rc) return rc;
+  const int cap = 16384;
+  const int tbytes = (64 + cap) * 4;
+  if (allow_smem(decode_tau_kernel, tbytes) != cudaSuccess) return NATTN_ECUDA;
+  decode_tau_kernel<<<rows, TAU_THREADS, tbytes, st>>>(A, const_cast<float*>(A.tau), cap);
+  if (check_launch()) return NATTN_ECUDA;
+  rc = launch_decode_mode<D, PS, DEC_APPLY>(a, A, mk, mv, st);
+  if (rc) return rc;
+  decode_combine_kernel<<<rows, 128, 0, st>>>(A, DEC_APPLY);
+  return check_launch();
+}
+
+int run(const nattn_args* a) {
+  int rc = validate(a);
+  if (rc != NATTN_OK) return rc;
+  if (a->B == 0 || a->Hq == 0 || a->Tq == 0) return NATTN_OK;
+  const Plan pl = make_plan(a);
+  if (pl.total > 0 && (a->workspace == nullptr || a->workspace_bytes < pl.total))
+    return NATTN_EWORKSPACE;
+  if (a->workspace && !aligned16(a->workspace)) return NATTN_EALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(a->stream);
+  const Problem P = to_problem(a);
+  uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+  switch (pl.path) {
+    case PATH_TC:
+      if (a->d == 64) return launch_tc<64>(a, P, pl, ws, st);
+      if (a->d == 128) return launch_tc<128>(a, P, pl, ws, st);
+      return launch_tc<256>(a, P, pl, ws, st);
+    case PATH_DECODE:
+      if (a->page_size == 32) {
+        if (a->d == 64) return launch_decode<64, 32>(a, P, pl, ws, st);
+        if (a->d == 128) return launch_decode<128, 32>(a, P, pl, ws, st);
+        return launch_decode<256, 32>(a, P, pl, ws, st);
+      }
+      if (a->d == 64) return launch_decode<64, 64>(a, P, pl, ws, st);
+      if (a->d == 128) return launch_decode<128, 64>(a, P, pl, ws, st);
+      return launch_decode<256, 64>(a, P, pl, ws, st);
+    case PATH_ROWWISE: {
+      const int nrows = a->B * a->Hq * a->Tq;
+      float* slots = pl.row_slots ? reinterpret_cast<float*>(ws + pl.off_slots) : nullptr;
+      return launch_rowwise(P, pl, nullptr, nullptr, nrows, slots, pl.row_grid, st);
+    }
+    default:
+      return NATTN_EUNSUPPORTED;
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+__attribute__((visibility("default"))) int nattn_fwd_ex(const nattn_args* a) { return run(a); }
+
+__attribute__((visibility("default"))) size_t nattn_workspace_size(const nattn_args* a) {
+  if (validate(a) != NATTN_OK) return 0;
+  if (a->B == 0 || a->Hq == 0 || a->Tq == 0) return 0;
+  return make_plan(a).total;
+}
+
+__attribute__((visibility("default"))) int nattn_fwd(const void* q, const void* k, const void* v, void* out, float* row_stat,
+              int B, int Hq, int Hkv, int Tq, int Tk, int d, int dv, float scale,
+              int normalizer, int causal, int window, float softcap,
+              const int32_t* block_table, const int32_t* seqlens, void* stream) {
+  nattn_args a;
+  memset(&a, 0, sizeof(a));
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.out = out;
+  a.row_stat = row_stat;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Tq = Tq;
+  a.Tk = Tk;
+  a.d = d;
+  a.dv = dv;
+  a.scale = scale;
+  a.normalizer = normalizer;
+  a.causal = causal;
+  a.window = window;
+  a.softcap = softcap;
+  a.block_table = block_table;
+  a.seqlens = seqlens;
+  a.stream = stream;
+  if (block_table) {
+    a.page_size = 64;
+    a.block_table_stride = (Tk + 63) / 64;
+    a.num_pages = 0x7fffffff / (Hkv > 0 ? Hkv * 64 : 64);
+  }
+  int rc = validate(&a);
+  if (rc != NATTN_OK) return rc;
+  const size_t need = nattn_workspace_size(&a);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (need > 0) {
+    if (cudaMallocAsync(&a.workspace, need, st) != cudaSuccess) return NATTN_ECUDA;
+    a.workspace_bytes = need;
+  }
+  rc = run(&a);
+  if (need > 0 && cudaFreeAsync(a.workspace, st) != cudaSuccess && rc == NATTN_OK)
+    rc = NATTN_ECUDA;
+  return rc;
+}
+
+__attribute__((visibility("default"))) int nattn_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return NATTN_ECUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return NATTN_ECUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return NATTN_ECUDA;
+  return v;
+}
+
+__attribute__((visibility("default"))) const char* nattn_strerror(int code) {
+  switch (code) {
+    case NATTN_OK: return "ok";
+    case NATTN_EINVAL: return "invalid argument";
+    case NATTN_EUNSUPPORTED: return "unsupported configuration";
+    case NATTN_ETOOLARGE: return "problem too large for the requested output";
+    case NATTN_EWORKSPACE: return "workspace missing or too small";
+    case NATTN_ECUDA: return "CUDA runtime error";
+    case NATTN_ETIMEOUT: return "device wait timed out";
+    case NATTN_EBOUNDS: return "block table entry or sequence length out of range";
+    case NATTN_EALIGN: return "pointer not 16-byte aligned";
+    default: return "unknown error";
+  }
+}
+
+__attribute__((visibility("default"))) int nattn_version(void) { return kVersion; }
+
+}  // extern "C"

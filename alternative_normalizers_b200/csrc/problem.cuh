@@ -1,0 +1,71 @@
+// The attention problem as the kernels see it, plus the two index rules
+// every kernel shares: which keys a query row may see, and where a key row
+// lives (dense tensor or paged pool).
+#pragma once
+
+#include "common.cuh"
+
+namespace nattn {
+
+struct Problem {
+  const bf16* q;
+  const bf16* k;
+  const bf16* v;
+  bf16* out;
+  float* row_stat;
+  float* weights;
+  int B, Hq, Hkv, Tq, Tk, d, dv;
+  float scale;
+  int norm;
+  int causal;
+  int window;
+  float softcap;
+  // paged mode (block_table != nullptr)
+  const int32_t* block_table;
+  const int32_t* seqlens;
+  int page_size, bt_stride, num_pages;
+};
+
+// Inclusive key range [lo, hi] visible to query row i when the row's key
+// length is L.  The query sits at key position pos = i + L - Tq (causal
+// diagonal aligned bottom-right, "HF Attention Normalizers", section "Packed
+// Variable-Length Attention").  Causal keeps j <= pos; a window W keeps
+// pos - j < W ("attention interface" wiki, "common flexattention patterns",
+// sliding window), and without causal also j - pos < W.  The visible set is
+// always one contiguous range (possibly empty: hi < lo).
+struct RowRange {
+  int lo, hi;
+};
+
+__host__ __device__ __forceinline__ RowRange row_range(int Tq, int causal, int window,
+                                                       int i, int L) {
+  const int pos = i + L - Tq;
+  int lo = 0, hi = L - 1;
+  if (causal && pos < hi) hi = pos;
+  if (window > 0) {
+    if (pos - window + 1 > lo) lo = pos - window + 1;
+    if (!causal && pos + window - 1 < hi) hi = pos + window - 1;
+  }
+  return RowRange{lo, hi};
+}
+
+__device__ __forceinline__ RowRange row_range(const Problem& P, int i, int L) {
+  return row_range(P.Tq, P.causal, P.window, i, L);
+}
+
+// Address of key (or value) row j of sequence b, kv head g.  Dense layout
+// [B, Hkv, Tk, dim]; paged pool [num_pages, Hkv, page_size, dim] through the
+// block table.  An out-of-range page id sets `bad` and returns nullptr.
+__device__ __forceinline__ const bf16* key_row(const Problem& P, const bf16* base, int dim,
+                                               int b, int g, int j, bool& bad) {
+  if (P.block_table == nullptr)
+    return base + (((size_t)b * P.Hkv + g) * P.Tk + j) * dim;
+  const int page = P.block_table[(size_t)b * P.bt_stride + j / P.page_size];
+  if (page < 0 || page >= P.num_pages) {
+    bad = true;
+    return nullptr;
+  }
+  return base + (((size_t)page * P.Hkv + g) * P.page_size + (j % P.page_size)) * dim;
+}
+
+}  // namespace nattn

@@ -1,0 +1,268 @@
+// Row-at-a-time attention on CUDA cores.
+//
+// One CTA owns one query row at a time: it materialises the row's allowed
+// scores (in shared memory, or in a per-CTA global slot for very long rows),
+// applies the row normalizer, optionally writes the dense weights, and
+// accumulates O = p V.  It serves three purposes:
+//   * the dense-weights request of the backend contract ("Attention",
+//     factory.ai transformers wiki: output plus optional weights),
+//   * small problems and head dims the tensor-core kernels do not take,
+//   * the sparse prefill rows whose support overflowed the phase-1 buffer.
+#pragma once
+
+#include "common.cuh"
+#include "problem.cuh"
+
+namespace nattn {
+
+constexpr int ROW_THREADS = 256;
+constexpr int ROW_WARPS = ROW_THREADS / 32;
+
+struct Red4 {
+  float a, b, c, d;
+};
+
+// Block-wide reduction of (sum, sum, sum, min).
+__device__ __forceinline__ Red4 block_red4(Red4 v, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v.a = warp_sum(v.a);
+  v.b = warp_sum(v.b);
+  v.c = warp_sum(v.c);
+  v.d = warp_min(v.d);
+  __syncthreads();
+  if (lane == 0) {
+    red[warp * 4 + 0] = v.a;
+    red[warp * 4 + 1] = v.b;
+    red[warp * 4 + 2] = v.c;
+    red[warp * 4 + 3] = v.d;
+  }
+  __syncthreads();
+  Red4 r{0.f, 0.f, 0.f, INFINITY};
+#pragma unroll
+  for (int w = 0; w < ROW_WARPS; ++w) {
+    r.a += red[w * 4 + 0];
+    r.b += red[w * 4 + 1];
+    r.c += red[w * 4 + 2];
+    r.d = fminf(r.d, red[w * 4 + 3]);
+  }
+  return r;
+}
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+  v = warp_max(v);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < ROW_WARPS; ++w) r = fmaxf(r, red[w]);
+  return r;
+}
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  v = warp_sum(v);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = 0.f;
+#pragma unroll
+  for (int w = 0; w < ROW_WARPS; ++w) r += red[w];
+  return r;
+}
+
+// Exact threshold of sparsemax / 1.5-entmax over sc[0..n) (values already in
+// threshold units u: z for sparsemax, z/2 for entmax), with u_max = m.
+//
+// Newton's method from the left on g(t) = sum relu(u - t)^k (k = 1 or 2),
+// which is convex and decreasing, so every iterate stays at or below the root
+// and the set {u > t} always contains the support.  At each iterate the
+// closed-form threshold of that set is tried first and accepted as soon as
+// it satisfies the optimality conditions (every member above it, every
+// other entry at or below it); for sparsemax this is Michelot's projection
+// algorithm.  Work is done in the shifted variable w = u - m for accuracy.
+__device__ float block_solve_tau(const float* sc, int n, float m, bool entmax,
+                                 float* red) {
+  float t = -1.0f;  // g(-1) >= 1 since the maximum contributes 1
+  for (int it = 0; it < 64; ++it) {
+    Red4 acc{0.f, 0.f, 0.f, INFINITY};
+    for (int j = threadIdx.x; j < n; j += ROW_THREADS) {
+      const float w = sc[j] - m;
+      if (w > t) {
+        acc.a += 1.f;
+        acc.b += w;
+        acc.c += w * w;
+        acc.d = fminf(acc.d, w);
+      }
+    }
+    const Red4 r = block_red4(acc, red);
+    const float cnt = r.a, s1 = r.b, s2 = r.c, wmin = r.d;
+    float ts, tn;
+    bool valid = true;
+    if (!entmax) {
+      ts = (s1 - 1.f) / cnt;
+      tn = ts;
+    } else {
+      const float mu = s1 / cnt;
+      const float delta = (1.f - (s2 - s1 * mu)) / cnt;
+      valid = delta >= 0.f;
+      ts = valid ? mu - sqrtf(delta) : -INFINITY;
+      const float g = s2 - 2.f * t * s1 + t * t * cnt;
+      const float gp = 2.f * (s1 - t * cnt);
+      tn = t + (g - 1.f) / gp;
+    }
+    if (valid && ts >= t && wmin > ts) {
+      t = ts;
+      break;
+    }
+    if (!(tn > t)) break;
+    t = tn;
+  }
+  return t + m;
+}
+
+// One CTA per query row (grid-stride over rows).  Dynamic shared memory:
+// q as float [256] | reduction scratch [64] | column partials [256] |
+// scores [cap].
+__global__ void __launch_bounds__(ROW_THREADS)
+    rowwise_kernel(Problem P, const int* __restrict__ row_list,
+                   const int* __restrict__ row_count, int nrows_static, int cap,
+                   float* __restrict__ gslots) {
+  extern __shared__ float smem_f[];
+  float* qf = smem_f;
+  float* red = qf + 256;
+  float* part = red + 64;
+  float* sc_smem = part + ROW_THREADS;
+  const int tid = threadIdx.x;
+  const int nrows = row_count ? *row_count : nrows_static;
+  const int group = P.Hq / P.Hkv;
+
+  for (int r = blockIdx.x; r < nrows; r += gridDim.x) {
+    const int flat = row_list ? row_list[r] : r;
+    const int i = flat % P.Tq;
+    const int h = (flat / P.Tq) % P.Hq;
+    const int b = flat / (P.Tq * P.Hq);
+    const int g = h / group;
+    int L = P.Tk;
+    bool bad = false;
+    if (P.block_table) {
+      L = P.seqlens[b];
+      if (L < 0 || L > P.Tk || L > P.bt_stride * P.page_size) bad = true;
+    }
+    const RowRange rr = row_range(P, i, bad ? 0 : L);
+    int n = rr.hi - rr.lo + 1;
+    if (n < 0) n = 0;
+    float* sc = sc_smem;
+    if (n > cap) {
+      if (gslots == nullptr) {
+        bad = true;
+        n = 0;
+      } else {
+        sc = gslots + (size_t)blockIdx.x * P.Tk;
+      }
+    }
+    bf16* orow = P.out + (size_t)flat * P.dv;
+    for (int c = tid; c < P.d; c += ROW_THREADS)
+      qf[c] = __bfloat162float(P.q[(size_t)flat * P.d + c]);
+    __syncthreads();
+
+    // scores z_j for the allowed keys, in units fixed by the normalizer
+    const float uscale = (P.norm == NATTN_ENTMAX15) ? 0.5f : 1.0f;
+    int badkey = 0;
+    for (int jj = tid; jj < n; jj += ROW_THREADS) {
+      const int j = rr.lo + jj;
+      bool kb = false;
+      const bf16* kp = key_row(P, P.k, P.d, b, g, j, kb);
+      float s = 0.f;
+      if (!kb) {
+        const uint4* k4 = reinterpret_cast<const uint4*>(kp);
+        for (int c8 = 0; c8 < P.d / 8; ++c8) {
+          const uint4 x = k4[c8];
+          const float* qq = qf + c8 * 8;
+          s += qq[0] * bf16lo(x.x) + qq[1] * bf16hi(x.x) + qq[2] * bf16lo(x.y) +
+               qq[3] * bf16hi(x.y) + qq[4] * bf16lo(x.z) + qq[5] * bf16hi(x.z) +
+               qq[6] * bf16lo(x.w) + qq[7] * bf16hi(x.w);
+        }
+      } else {
+        badkey = 1;
+      }
+      float z = s * P.scale;
+      if (P.softcap > 0.f) z = P.softcap * tanhf(z / P.softcap);
+      sc[jj] = z * uscale;
+    }
+    if (__syncthreads_or(badkey)) bad = true;
+    if (bad) {
+      set_status(NATTN_EBOUNDS);
+      n = 0;
+    }
+
+    // normalizer: overwrite scores with weights
+    float stat;
+    if (P.norm == NATTN_SOFTMAX || P.norm == NATTN_SOFTMAX1) {
+      float mx = -INFINITY;
+      for (int jj = tid; jj < n; jj += ROW_THREADS) mx = fmaxf(mx, sc[jj]);
+      mx = block_max(mx, red);
+      if (P.norm == NATTN_SOFTMAX1) mx = fmaxf(mx, 0.f);
+      const float msafe = (mx == -INFINITY) ? 0.f : mx;
+      float l = 0.f;
+      for (int jj = tid; jj < n; jj += ROW_THREADS) {
+        const float e = expf(sc[jj] - msafe);
+        sc[jj] = e;
+        l += e;
+      }
+      l = block_sum(l, red);
+      if (P.norm == NATTN_SOFTMAX1) l += expf(-msafe);
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      for (int jj = tid; jj < n; jj += ROW_THREADS) sc[jj] *= inv;
+      stat = (l > 0.f) ? msafe + logf(l) : -INFINITY;
+    } else {
+      const bool ent = P.norm == NATTN_ENTMAX15;
+      float mx = -INFINITY;
+      for (int jj = tid; jj < n; jj += ROW_THREADS) mx = fmaxf(mx, sc[jj]);
+      mx = block_max(mx, red);
+      float tau = INFINITY;
+      if (n > 0) tau = block_solve_tau(sc, n, mx, ent, red);
+      __syncthreads();
+      for (int jj = tid; jj < n; jj += ROW_THREADS) {
+        const float t = fmaxf(sc[jj] - tau, 0.f);
+        sc[jj] = ent ? t * t : t;
+      }
+      stat = tau;
+    }
+    __syncthreads();
+
+    if (P.weights) {
+      float* wrow = P.weights + (size_t)flat * P.Tk;
+      for (int j = tid; j < P.Tk; j += ROW_THREADS) {
+        const int jj = j - rr.lo;
+        wrow[j] = (jj >= 0 && jj < n) ? sc[jj] : 0.f;
+      }
+    }
+
+    // O = p V: thread (grp, c) sums keys grp, grp + G, ... for column c
+    const int G = ROW_THREADS / P.dv;
+    const int c = tid % P.dv, grp = tid / P.dv;
+    float acc = 0.f;
+    if (grp < G) {
+      for (int jj = grp; jj < n; jj += G) {
+        const float p = sc[jj];
+        if (p != 0.f) {
+          bool kb = false;
+          const bf16* vp = key_row(P, P.v, P.dv, b, g, rr.lo + jj, kb);
+          acc += p * __bfloat162float(vp[c]);
+        }
+      }
+    }
+    __syncthreads();
+    if (grp < G) part[grp * P.dv + c] = acc;
+    __syncthreads();
+    if (tid < P.dv) {
+      float o = 0.f;
+      for (int q2 = 0; q2 < G; ++q2) o += part[q2 * P.dv + tid];
+      orow[tid] = __float2bfloat16_rn(o);
+    }
+    if (tid == 0 && P.row_stat) P.row_stat[flat] = stat;
+    __syncthreads();
+  }
+}
+
+}  // namespace nattn

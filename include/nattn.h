@@ -1,0 +1,177 @@
+/*
+ * libnattn: fused attention forward with a selectable row normalizer, for
+ * NVIDIA B200 (sm_100a).
+ *
+ *     O = N(scale * Q K^T + mask) V
+ *
+ * The backend contract follows "Attention" (factory.ai transformers wiki),
+ * section "What every backend must support": query, key and value after
+ * grouped-query expansion, a mask, the scaling factor and is_causal in; the
+ * attention output and, on request, the attention weights out.  Here the
+ * grouped-query expansion is done inside the kernels (key/value heads are
+ * passed unexpanded, query head h reads key/value head h / (Hq / Hkv)).
+ *
+ * The normalizers are those of "HF Attention Normalizers" (PyPI project
+ * page), section "Supported Normalizers":
+ *   NATTN_SOFTMAX    exp(z_i) / sum_j exp(z_j)
+ *   NATTN_SOFTMAX1   exp(z_i) / (1 + sum_j exp(z_j))   (Softmax-N, n = 1)
+ *   NATTN_SPARSEMAX  Euclidean projection onto the probability simplex,
+ *                    p_i = max(z_i - tau, 0)
+ *   NATTN_ENTMAX15   1.5-entmax, p_i = max(z_i / 2 - tau, 0)^2
+ *
+ * The mask switches are those of the "sdpa" primitive in "Attention variants:
+ * what to open up, and how far" (TensorCAD), section "What the engine does
+ * today": causal, sliding window, and the Gemma-2 logit soft-cap
+ * cap * tanh(score / cap).  Scores are scaled, then capped, then masked.
+ *
+ * Conventions for every entry point:
+ *   - All tensors are contiguous, row-major, in device memory, and start on a
+ *     16-byte boundary.  Q/K/V/O are bfloat16; row_stat and weights float32;
+ *     block tables and sequence lengths int32.
+ *   - The caller owns every buffer.  nattn_fwd_ex allocates nothing; nattn_fwd
+ *     allocates stream-ordered scratch (cudaMallocAsync / cudaFreeAsync on
+ *     the given stream) only when the chosen path needs it.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and return after launching.  Errors found on the host
+ *     are returned before anything is launched; errors found on the device
+ *     (a bad block-table entry, a bounded wait that gave up) are recorded in a
+ *     per-device status word read by nattn_get_device_status().
+ *   - There is no fallback: an unsupported request returns an error code and
+ *     computes nothing ("HF Attention Normalizers", section "Strict vs
+ *     Fallback Mode": strict mode raises a clear error).
+ */
+#ifndef NATTN_H
+#define NATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NATTN_SOFTMAX = 0,
+  NATTN_SOFTMAX1 = 1,
+  NATTN_SPARSEMAX = 2,
+  NATTN_ENTMAX15 = 3
+} nattn_normalizer;
+
+enum {
+  NATTN_OK = 0,
+  NATTN_EINVAL = -1,        /* bad argument: NULL pointer, negative size,
+                               Hq % Hkv != 0, non-finite scale, ...        */
+  NATTN_EUNSUPPORTED = -2,  /* well-formed but outside what the kernels do:
+                               head dim not in {32, 64, 128, 256}, paged mode
+                               with dense weights, ...                       */
+  NATTN_ETOOLARGE = -3,     /* dense weights asked for more than 2^26 entries,
+                               or a size beyond the int32 index range       */
+  NATTN_EWORKSPACE = -4,    /* workspace NULL or smaller than
+                               nattn_workspace_size()                        */
+  NATTN_ECUDA = -5,         /* a CUDA runtime call or kernel launch failed  */
+  NATTN_ETIMEOUT = -6,      /* device: a bounded wait gave up               */
+  NATTN_EBOUNDS = -7,       /* device: a block-table entry or a sequence
+                               length was out of range; the offending work
+                               item wrote zeros and was skipped             */
+  NATTN_EALIGN = -8         /* a pointer is not 16-byte aligned             */
+};
+
+/*
+ * Full argument block.
+ *
+ * Dense mode (block_table == NULL):
+ *   q        bf16 [B, Hq, Tq, d]
+ *   k        bf16 [B, Hkv, Tk, d]
+ *   v        bf16 [B, Hkv, Tk, dv]
+ *   Query row i sits at key position i + (Tk - Tq) (causal mask aligned
+ *   bottom-right, "HF Attention Normalizers", section "Packed Variable-Length
+ *   Attention").
+ *
+ * Paged mode (block_table != NULL), the paged KV cache of "HF Attention
+ * Normalizers", section "Differentiable Paged Attention" (key_cache,
+ * value_cache, block_table, sequence_lengths, block_size):
+ *   q        bf16 [B, Hq, Tq, d]   (Tq new tokens per sequence; decode: 1)
+ *   k        bf16 [num_pages, Hkv, page_size, d]   physical page pool
+ *   v        bf16 [num_pages, Hkv, page_size, dv]
+ *   block_table  int32 [B, block_table_stride]: logical page p of sequence b
+ *                lives in physical page block_table[b * stride + p]
+ *   seqlens  int32 [B]: key length of each sequence, 1 <= seqlens[b] <= Tk
+ *   Tk       the largest key length any sequence may have (sizes scratch)
+ *   Query row i of sequence b sits at key position i + seqlens[b] - Tq.
+ *
+ * Outputs (both modes):
+ *   out      bf16 [B, Hq, Tq, dv]  (rows with no visible key are all zero)
+ *   row_stat float32 [B, Hq, Tq] or NULL.  softmax: natural-log
+ *            log-sum-exp (-inf for a row with no visible key); softmax1:
+ *            log(1 + sum exp z) (0 for such a row); sparsemax: tau; entmax15:
+ *            tau in units of z/2 (+inf for such a row).
+ *   weights  float32 [B, Hq, Tq, Tk] dense attention weights or NULL (dense
+ *            mode only, at most 2^26 entries; masked entries are exactly 0).
+ *
+ * window == 0 disables the sliding window; with causal it keeps keys with
+ * 0 <= pos - j < window ("attention interface" wiki, section "common
+ * flexattention patterns"); without causal it keeps |pos - j| < window.
+ * softcap == 0 disables the soft-cap.
+ */
+typedef struct nattn_args {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  float* row_stat;
+  float* weights;
+  int B, Hq, Hkv, Tq, Tk, d, dv;
+  float scale;
+  int normalizer;
+  int causal;
+  int window;
+  float softcap;
+  const int32_t* block_table;
+  const int32_t* seqlens;
+  int page_size;
+  int block_table_stride;
+  int num_pages;
+  void* workspace;          /* device scratch, >= nattn_workspace_size(args) */
+  size_t workspace_bytes;
+  void* stream;             /* cudaStream_t */
+} nattn_args;
+
+/*
+ * Attention forward with the argument list of the backend contract.
+ * Dense mode when block_table == NULL.  In paged mode this short form fixes
+ * page_size = 64, block_table_stride = ceil(Tk / 64) and does not bound the
+ * page ids from above (use nattn_fwd_ex for other layouts).  Scratch the
+ * chosen path needs is allocated and freed stream-ordered on `stream`.
+ * Returns NATTN_OK or a negative error code.
+ */
+int nattn_fwd(const void* q, const void* k, const void* v, void* out,
+              float* row_stat, int B, int Hq, int Hkv, int Tq, int Tk, int d,
+              int dv, float scale, int normalizer, int causal, int window,
+              float softcap, const int32_t* block_table,
+              const int32_t* seqlens, void* stream);
+
+/* Attention forward from a full argument block; allocates nothing.  The
+ * caller passes scratch of at least nattn_workspace_size(a) bytes (NULL is
+ * fine when that size is 0).  Returns NATTN_OK or a negative error code. */
+int nattn_fwd_ex(const nattn_args* a);
+
+/* Bytes of device scratch nattn_fwd_ex needs for these arguments (pointers
+ * are not read).  Returns 0 for an invalid argument block. */
+size_t nattn_workspace_size(const nattn_args* a);
+
+/* Synchronises `stream`, returns the device status word of the current device
+ * (NATTN_OK, NATTN_ETIMEOUT or NATTN_EBOUNDS; the first error recorded since
+ * the last call wins) and clears it.  NATTN_ECUDA if the sync itself fails. */
+int nattn_get_device_status(void* stream);
+
+/* Static description of an error code. */
+const char* nattn_strerror(int code);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int nattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NATTN_H */
