@@ -12,7 +12,7 @@ import os
 from .workloads import NORMALIZER_IDS
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "lib", "libnattn.so")
+LIB_PATH = os.environ.get("NATTN_LIB") or os.path.join(_HERE, "lib", "libnattn.so")
 
 NATTN_OK = 0
 ERRORS = {

@@ -58,7 +58,9 @@ struct DecodeSmem {
   static constexpr int PSTRIDE = PS * 2 + 16;        // bytes per P row
   static constexpr int OFF_S = NS * STAGE;
   static constexpr int OFF_P = OFF_S + 16 * SSTRIDE * 4;
-  static constexpr int OFF_A = OFF_P + 16 * PSTRIDE;
+  // APPLY keeps P as bf16 hi + lo planes (weights to ~16 mantissa bits)
+  static constexpr int OFF_PL = OFF_P + 16 * PSTRIDE;
+  static constexpr int OFF_A = OFF_PL + ((MODE == DEC_APPLY) ? 16 * PSTRIDE : 0);
   static constexpr int OFF_BAR = OFF_A + 16 * 4;
   static constexpr int OFF_FLAGS = OFF_BAR + NS * 8;
   static constexpr int OFF_LIST = OFF_FLAGS + NS * 4;
@@ -115,6 +117,7 @@ __global__ void __launch_bounds__(DEC_THREADS)
 
   float* S = reinterpret_cast<float*>(smem + L::OFF_S);
   uint8_t* Pb = smem + L::OFF_P;
+  uint8_t* Pl = smem + L::OFF_PL;
   float* alpha = reinterpret_cast<float*>(smem + L::OFF_A);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   int* badflag = reinterpret_cast<int*>(smem + L::OFF_FLAGS);
@@ -212,7 +215,7 @@ __global__ void __launch_bounds__(DEC_THREADS)
     for (int e = 0; e < 4; ++e) oacc[n][e] = 0.f;
 
   // zero the unused P rows once (rows >= R stay zero)
-  for (int x = tid; x < 16 * L::PSTRIDE / 4; x += DEC_THREADS)
+  for (int x = tid; x < (L::OFF_A - L::OFF_P) / 4; x += DEC_THREADS)
     reinterpret_cast<uint32_t*>(Pb)[x] = 0u;
   __syncthreads();
 
@@ -343,7 +346,10 @@ __global__ void __launch_bounds__(DEC_THREADS)
             const float x = fmaxf(u - tr, 0.f);
             w = (P.norm == NATTN_ENTMAX15) ? x * x : x;
           }
-          reinterpret_cast<bf16*>(Pb + r * L::PSTRIDE)[jj] = __float2bfloat16_rn(w);
+          const bf16 wh = __float2bfloat16_rn(w);
+          reinterpret_cast<bf16*>(Pb + r * L::PSTRIDE)[jj] = wh;
+          reinterpret_cast<bf16*>(Pl + r * L::PSTRIDE)[jj] =
+              __float2bfloat16_rn(w - __bfloat162float(wh));
         }
       }
       __syncthreads();
@@ -366,11 +372,13 @@ __global__ void __launch_bounds__(DEC_THREADS)
       const int col0 = warp * (DV / 4);
 #pragma unroll
       for (int kk = 0; kk < PS / 16; ++kk) {
-        uint32_t a0, a1, a2, a3;
+        uint32_t a0, a1, a2, a3, l0 = 0, l1 = 0, l2 = 0, l3 = 0;
         {
           const int prow = (lane & 7) + 8 * ((lane >> 3) & 1);
           const int pchunk = kk * 2 + (lane >> 4);
           ldsm_x4(smem_addr(Pb + prow * L::PSTRIDE + pchunk * 16), a0, a1, a2, a3);
+          if constexpr (MODE == DEC_APPLY)
+            ldsm_x4(smem_addr(Pl + prow * L::PSTRIDE + pchunk * 16), l0, l1, l2, l3);
         }
 #pragma unroll
         for (int n = 0; n < NOT; n += 2) {
@@ -381,6 +389,10 @@ __global__ void __launch_bounds__(DEC_THREADS)
                     b1, b2, b3);
           mma_bf16_16816(oacc[n], a0, a1, a2, a3, b0, b1);
           if (n + 1 < NOT) mma_bf16_16816(oacc[n + 1], a0, a1, a2, a3, b2, b3);
+          if constexpr (MODE == DEC_APPLY) {
+            mma_bf16_16816(oacc[n], l0, l1, l2, l3, b0, b1);
+            if (n + 1 < NOT) mma_bf16_16816(oacc[n + 1], l0, l1, l2, l3, b2, b3);
+          }
         }
       }
     }

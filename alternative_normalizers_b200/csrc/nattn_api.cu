@@ -22,7 +22,6 @@ using namespace nattn;
 namespace {
 
 constexpr int kVersion = 100;  // 0.1.0
-constexpr int kMaxDevices = 64;
 constexpr int kRowSmemCap = 48 * 1024;  // scores kept in shared memory per row
 constexpr long long kMaxWeights = 1ll << 26;
 
@@ -100,6 +99,9 @@ struct Plan {
   int R = 0, nsplit = 0, pps = 0;
   // scratch offsets (bytes)
   size_t off_tau = 0, off_ovfc = 0, off_ovfr = 0, off_slots = 0;
+  size_t off_supc = 0, off_supl = 0;
+  int sup_cap = 0;
+  bool tc_apply = false;  // sparse phase 2 on the tensor cores (bf16 P)
   size_t off_opart = 0, off_ml = 0, off_scores = 0;
   size_t total = 0;
   int row_grid = 0, row_cap = 0;
@@ -190,6 +192,15 @@ Plan make_plan(const nattn_args* a) {
       off = up256(off + 4);
       pl.off_ovfr = off;
       off = up256(off + rows * 4);
+      pl.sup_cap = (a->d >= 256) ? TauCap<256>::value : TauCap<128>::value;
+      pl.off_supc = off;
+      off = up256(off + rows * 4);
+      pl.off_supl = off;
+      off = up256(off + rows * (size_t)pl.sup_cap * 8);
+      {
+        const char* e = getenv("NATTN_SPARSE_APPLY");
+        pl.tc_apply = e && strcmp(e, "tc") == 0;
+      }
       pl.row_grid = 2 * 148;
       pl.row_cap = a->Tk < kRowSmemCap ? (a->Tk < 256 ? 256 : a->Tk) : kRowSmemCap;
       if (a->Tk > kRowSmemCap) {
@@ -281,6 +292,9 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
     A.tau = nullptr;
     A.ovf_rows = nullptr;
     A.ovf_count = nullptr;
+    A.sup_count = nullptr;
+    A.sup_list = nullptr;
+    A.sup_cap = 0;
     using LY = TcLayout<D, D, BN, KST, VST, TC_ONLINE>;
     auto k = prefill_tc_kernel<D, D, BN, KST, VST, TC_ONLINE>;
     if (allow_smem(k, LY::ALLOC) != cudaSuccess) return NATTN_ECUDA;
@@ -293,19 +307,28 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
   A.tau = reinterpret_cast<float*>(ws + pl.off_tau);
   A.ovf_count = reinterpret_cast<int*>(ws + pl.off_ovfc);
   A.ovf_rows = reinterpret_cast<int*>(ws + pl.off_ovfr);
+  A.sup_count = reinterpret_cast<int*>(ws + pl.off_supc);
+  A.sup_list = reinterpret_cast<int2*>(ws + pl.off_supl);
+  A.sup_cap = pl.sup_cap;
   if (cudaMemsetAsync(A.ovf_count, 0, sizeof(int), st) != cudaSuccess) return NATTN_ECUDA;
   {
-    using LY = TcLayout<D, D, BN, 3, 1, TC_TAU>;
-    auto k = prefill_tc_kernel<D, D, BN, 3, 1, TC_TAU>;
+    using LY = TcLayout<D, D, BN, 2, 1, TC_TAU>;
+    auto k = prefill_tc_kernel<D, D, BN, 2, 1, TC_TAU>;
     if (allow_smem(k, LY::ALLOC) != cudaSuccess) return NATTN_ECUDA;
     k<<<grid, TC_THREADS, LY::ALLOC, st>>>(mq, mk, mv, A);
     if (check_launch() != NATTN_OK) return NATTN_ECUDA;
   }
-  {
+  if (pl.tc_apply) {
     using LY = TcLayout<D, D, BN, KST, VST, TC_APPLY>;
     auto k = prefill_tc_kernel<D, D, BN, KST, VST, TC_APPLY>;
     if (allow_smem(k, LY::ALLOC) != cudaSuccess) return NATTN_ECUDA;
     k<<<grid, TC_THREADS, LY::ALLOC, st>>>(mq, mk, mv, A);
+    if (check_launch() != NATTN_OK) return NATTN_ECUDA;
+  } else {
+    const size_t rows = (size_t)a->B * a->Hq * a->Tq;
+    const unsigned g2 = (unsigned)((rows + GATHER_WARPS - 1) / GATHER_WARPS);
+    sparse_gather_kernel<D><<<g2, GATHER_WARPS * 32, 0, st>>>(P, A.sup_count, A.sup_list,
+                                                              A.sup_cap, A.tau);
     if (check_launch() != NATTN_OK) return NATTN_ECUDA;
   }
   // rows whose candidate buffer overflowed: exact row-wise recomputation

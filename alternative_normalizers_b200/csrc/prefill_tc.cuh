@@ -47,7 +47,11 @@ enum TcMode { TC_ONLINE = 0, TC_TAU = 1, TC_APPLY = 2 };
 
 constexpr int TC_THREADS = 192;
 constexpr int TC_BM = 128;
-constexpr int TAU_CAP = 128;  // candidate buffer entries per row
+// candidate buffer entries per row in the threshold pass (value + key index)
+template <int D>
+struct TauCap {
+  static constexpr int value = (D >= 256) ? 64 : 128;
+};
 
 struct TcArgs {
   Problem P;
@@ -56,6 +60,9 @@ struct TcArgs {
   float* tau;        // [B*Hq*Tq]: written by TAU, read by APPLY
   int* ovf_rows;     // TAU: rows whose candidate buffer overflowed
   int* ovf_count;    // TAU: number of such rows (zeroed before the launch)
+  int* sup_count;    // TAU: support size of every row (0 for overflowed rows)
+  int2* sup_list;    // TAU: [rows][sup_cap] (key index, weight bits)
+  int sup_cap;
 };
 
 template <int D, int DV, int BN, int KST, int VST, int MODE>
@@ -67,7 +74,9 @@ struct TcLayout {
   static constexpr int OFF_K = OFF_Q + QBYTES;
   static constexpr int OFF_V = OFF_K + KST * KBYTES;
   static constexpr int OFF_BUF = OFF_V + VST * VBYTES;
-  static constexpr int BUFBYTES = (MODE == TC_TAU) ? TAU_CAP * TC_BM * 4 : 0;
+  static constexpr int CAP = TauCap<D>::value;
+  static constexpr int BUFBYTES = (MODE == TC_TAU) ? 2 * CAP * TC_BM * 4 : 0;
+  static constexpr int OFF_IDX = OFF_BUF + CAP * TC_BM * 4;
   static constexpr int OFF_BAR = OFF_BUF + BUFBYTES;
   static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 2 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -99,7 +108,7 @@ __device__ __forceinline__ float tc_z(float s, const TcArgs& A) {
 // threshold of {u > t} once it satisfies the optimality conditions.
 // `t0` is a lower bound of tau in shifted units (u - m).  With `newton_only`
 // it returns after `iters` Newton steps (a valid lower bound, for pruning).
-__device__ __forceinline__ float thread_tau(const float* buf, int n, float m, bool entmax,
+__device__ __noinline__ float thread_tau(const float* buf, int n, float m, bool entmax,
                                             float t0, int iters, bool newton_only) {
   float t = fmaxf(t0, -1.f);
   for (int it = 0; it < iters; ++it) {
@@ -187,7 +196,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar_sfull(s), 1);
-      mbar_init(bar_pfull(s), 128);
+      mbar_init(bar_pfull(s), 4);
     }
     mbar_init(bar_pv, 1);
     *abort_flag = 0;
@@ -302,10 +311,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (rr.hi > P.Tk - 1) rr.hi = P.Tk - 1;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     const size_t flat = ((size_t)bh * P.Tq + qi);
+    // fast path: no soft-cap and a positive scale, so max(z) = scale * max(s)
+    // and exp2(z - m) is one FFMA + EX2 per score
+    const bool fast = !(P.softcap > 0.f) && A.zscale > 0.f;
+    const float zs = A.zscale;
 
     float m_run, l_run = 0.f, tau = 0.f;
     // TAU state
     float* buf = reinterpret_cast<float*>(smem + LY::OFF_BUF) + row;
+    int* bidx = reinterpret_cast<int*>(smem + LY::OFF_IDX) + row;
     int nbuf = 0;
     bool ovf = false;
     float lb = -INFINITY;  // lower bound of tau (threshold units)
@@ -328,57 +342,68 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tc_fence_after();
       const int j0 = (kb0 + j) * BN;
       const bool edge = !(rr.lo <= j0 && rr.hi >= j0 + BN - 1);
+      // visible keys of this row inside the block: [kl, kl + span]
+      int kl = rr.lo - j0;
+      unsigned span = (unsigned)(rr.hi - rr.lo);
+      if (rr.hi < rr.lo) {
+        kl = BN;
+        span = 0;
+      }
       const uint32_t saddr = lane_base + (sb ? LY::TM_S1 : LY::TM_S0);
 
-      if constexpr (MODE == TC_ONLINE) {
-        // pass 1: row maximum of this block
-        float mx = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(saddr + c * 32, r);
-          tmem_ld_wait();
+      // the whole S row of this block, one TMEM round trip
+      uint32_t r[BN];
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            float z = tc_z(__uint_as_float(r[k]), A);
-            if (edge) {
-              const int jj = j0 + c * 32 + k;
-              z = (jj >= rr.lo && jj <= rr.hi) ? z : -INFINITY;
-            }
-            mx = fmaxf(mx, z);
-          }
+      for (int c = 0; c < BN / 32; ++c)
+        tmem_ld32(saddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+      tmem_ld_wait();
+
+      // scores -> z (threshold / log2 units) unless the fast path keeps raw s;
+      // masked entries become -inf
+      if (!fast) {
+#pragma unroll
+        for (int k = 0; k < BN; ++k) r[k] = __float_as_uint(tc_z(__uint_as_float(r[k]), A));
+      }
+      if (edge) {
+#pragma unroll
+        for (int k = 0; k < BN; ++k)
+          if ((unsigned)(k - kl) > span) r[k] = __float_as_uint(-INFINITY);
+      }
+
+      if constexpr (MODE == TC_ONLINE) {
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < BN; k += 4) {
+          mx0 = fmaxf(mx0, __uint_as_float(r[k]));
+          mx1 = fmaxf(mx1, __uint_as_float(r[k + 1]));
+          mx2 = fmaxf(mx2, __uint_as_float(r[k + 2]));
+          mx3 = fmaxf(mx3, __uint_as_float(r[k + 3]));
         }
+        float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        if (fast) mx *= zs;
         const float mnew = fmaxf(m_run, mx);
         const bool resc = mnew > m_run + 8.f;
         const float m_use = resc ? mnew : m_run;
         const float alpha = resc ? fast_exp2(m_run - mnew) : 1.f;
         const float msafe = (m_use == -INFINITY) ? 0.f : m_use;
-        // pass 2: weights, row sum, bf16 P into the S columns
-        float sum = 0.f;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(saddr + c * 32, r);
-          tmem_ld_wait();
-          uint32_t pk[16];
+        const float fa = fast ? zs : 1.f;  // p = exp2(x * fa - msafe)
+        float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            float z0 = tc_z(__uint_as_float(r[k]), A);
-            float z1 = tc_z(__uint_as_float(r[k + 1]), A);
-            if (edge) {
-              const int jj = j0 + c * 32 + k;
-              z0 = (jj >= rr.lo && jj <= rr.hi) ? z0 : -INFINITY;
-              z1 = (jj + 1 >= rr.lo && jj + 1 <= rr.hi) ? z1 : -INFINITY;
-            }
-            const float p0 = fast_exp2(z0 - msafe);
-            const float p1 = fast_exp2(z1 - msafe);
-            sum += p0 + p1;
+        for (int c = 0; c < BN / 64; ++c) {  // 64 scores -> 32 packed columns
+          uint32_t pk[32];
+#pragma unroll
+          for (int k = 0; k < 64; k += 2) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(r[c * 64 + k]), fa, -msafe));
+            const float p1 =
+                fast_exp2(fmaf(__uint_as_float(r[c * 64 + k + 1]), fa, -msafe));
+            s0 += p0;
+            s1 += p1;
             pk[k >> 1] = pack_bf16(p0, p1);
           }
-          tmem_st16(saddr + c * 16, pk);
+          tmem_st32(saddr + c * 32, pk);
         }
         tmem_st_wait();
-        l_run = l_run * alpha + sum;
+        l_run = l_run * alpha + (s0 + s1);
         // rescale O when the maximum moved (warp-uniform TMEM access)
         if (__any_sync(0xffffffffu, resc) && j > 0) {
           if (!__all_sync(0xffffffffu, mbar_wait(bar_pv, (j - 1) & 1, abort_flag))) {
@@ -389,77 +414,67 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           const uint32_t oaddr = lane_base + LY::TM_O;
 #pragma unroll 1
           for (int c = 0; c < DV / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(oaddr + c * 32, r);
+            uint32_t o[32];
+            tmem_ld32(oaddr + c * 32, o);
             tmem_ld_wait();
 #pragma unroll
-            for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
-            tmem_st32(oaddr + c * 32, r);
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st32(oaddr + c * 32, o);
           }
           tmem_st_wait();
         }
         m_run = m_use;
       } else if constexpr (MODE == TC_APPLY) {
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(saddr + c * 32, r);
-          tmem_ld_wait();
-          uint32_t pk[16];
+        // p = relu(z - tau) or relu(z/2 - tau)^2 as bf16 P
+        const float fa = fast ? zs : 1.f;
 #pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            float x0 = fmaxf(tc_z(__uint_as_float(r[k]), A) - tau, 0.f);
-            float x1 = fmaxf(tc_z(__uint_as_float(r[k + 1]), A) - tau, 0.f);
+        for (int c = 0; c < BN / 64; ++c) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int k = 0; k < 64; k += 2) {
+            float x0 = fmaxf(fmaf(__uint_as_float(r[c * 64 + k]), fa, -tau), 0.f);
+            float x1 = fmaxf(fmaf(__uint_as_float(r[c * 64 + k + 1]), fa, -tau), 0.f);
             if (entmax) {
               x0 *= x0;
               x1 *= x1;
             }
-            if (edge) {
-              const int jj = j0 + c * 32 + k;
-              x0 = (jj >= rr.lo && jj <= rr.hi) ? x0 : 0.f;
-              x1 = (jj + 1 >= rr.lo && jj + 1 <= rr.hi) ? x1 : 0.f;
-            }
             pk[k >> 1] = pack_bf16(x0, x1);
           }
-          tmem_st16(saddr + c * 16, pk);
+          tmem_st32(saddr + c * 32, pk);
         }
         tmem_st_wait();
       } else {  // TC_TAU
-#pragma unroll 1
+#pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(saddr + c * 32, r);
-          tmem_ld_wait();
-          float u[32];
           float cmax = -INFINITY;
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
-            float z = tc_z(__uint_as_float(r[k]), A);
-            if (edge) {
-              const int jj = j0 + c * 32 + k;
-              z = (jj >= rr.lo && jj <= rr.hi) ? z : -INFINITY;
-            }
-            u[k] = z;
-            cmax = fmaxf(cmax, z);
+            if (fast) r[c * 32 + k] = __float_as_uint(__uint_as_float(r[c * 32 + k]) * zs);
+            cmax = fmaxf(cmax, __uint_as_float(r[c * 32 + k]));
           }
           m_run = fmaxf(m_run, cmax);
           lb = fmaxf(lb, m_run - 1.f);  // tau >= max - 1
           if (cmax > lb && !ovf) {
-            if (nbuf + 32 > TAU_CAP) {
+            if (nbuf + 32 > LY::CAP) {
               // raise the lower bound with a few Newton steps, then compact
               lb = thread_tau(buf, nbuf, m_run, entmax, lb - m_run, 4, true);
               int w = 0;
               for (int k = 0; k < nbuf; ++k) {
                 const float x = buf[k * TC_BM];
-                if (x > lb) buf[(w++) * TC_BM] = x;
+                if (x > lb) {
+                  bidx[w * TC_BM] = bidx[k * TC_BM];
+                  buf[(w++) * TC_BM] = x;
+                }
               }
               nbuf = w;
             }
 #pragma unroll
             for (int k = 0; k < 32; ++k) {
-              if (u[k] > lb) {
-                if (nbuf < TAU_CAP) {
-                  buf[nbuf * TC_BM] = u[k];
+              const float u = __uint_as_float(r[c * 32 + k]);
+              if (u > lb) {
+                if (nbuf < LY::CAP) {
+                  buf[nbuf * TC_BM] = u;
+                  bidx[nbuf * TC_BM] = j0 + c * 32 + k;
                   ++nbuf;
                 } else {
                   ovf = true;
@@ -470,20 +485,32 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar_pfull(sb));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_pfull(sb));
     }
 
     // ---- epilogue ----------------------------------------------------------
     if constexpr (MODE == TC_TAU) {
       if (row_ok) {
         float t = INFINITY;
+        int nsup = 0;
         if (ovf) {
           const int slot = atomicAdd(A.ovf_count, 1);
           A.ovf_rows[slot] = (int)flat;
         } else if (m_run != -INFINITY) {
           t = thread_tau(buf, nbuf, m_run, entmax, lb - m_run, 64, false);
+          // the support and its weights, for the gather pass
+          int2* dst = A.sup_list + flat * (size_t)A.sup_cap;
+          for (int k = 0; k < nbuf; ++k) {
+            const float x = buf[k * TC_BM] - t;
+            if (x > 0.f) {
+              const float w = entmax ? x * x : x;
+              dst[nsup++] = make_int2(bidx[k * TC_BM], __float_as_int(w));
+            }
+          }
         }
         A.tau[flat] = t;
+        A.sup_count[flat] = nsup;
       }
     } else {
       const bool have_o =
@@ -529,6 +556,66 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 5) tmem_dealloc(tmem, LY::TM_COLS);
+}
+
+
+// Sparse phase 2 (default): O = sum over the row's support of p_j V_j, in
+// fp32 on CUDA cores, from the (key, weight) list the threshold pass wrote.
+// The support of sparsemax / 1.5-entmax is a handful of keys per row, so
+// this touches |support| value rows instead of multiplying every block, and
+// the weights enter the sum in full precision.  One warp per query row; lane
+// l owns columns [l * dv/32, (l+1) * dv/32).
+constexpr int GATHER_WARPS = 4;
+
+template <int DV>
+__global__ void __launch_bounds__(GATHER_WARPS * 32)
+    sparse_gather_kernel(Problem P, const int* __restrict__ sup_count,
+                         const int2* __restrict__ sup_list, int sup_cap,
+                         const float* __restrict__ tau) {
+  constexpr int PER = DV / 32;  // columns per lane (2, 4 or 8)
+  const int lane = threadIdx.x & 31;
+  const size_t rows = (size_t)P.B * P.Hq * P.Tq;
+  const size_t flat = (size_t)blockIdx.x * GATHER_WARPS + (threadIdx.x >> 5);
+  if (flat >= rows) return;
+  const int h = (int)((flat / P.Tq) % P.Hq);
+  const int b = (int)(flat / ((size_t)P.Tq * P.Hq));
+  const int g = h / (P.Hq / P.Hkv);
+  const int n = sup_count[flat];
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  if (n > 0) {
+    const bf16* vbase = P.v + ((size_t)b * P.Hkv + g) * (size_t)P.Tk * DV + lane * PER;
+    const int2* lst = sup_list + flat * (size_t)sup_cap;
+    for (int e0 = 0; e0 < n; e0 += 32) {
+      const int2 mine = (e0 + lane < n) ? lst[e0 + lane] : make_int2(0, 0);
+      const int cnt = min(32, n - e0);
+      for (int e = 0; e < cnt; ++e) {
+        const int j = __shfl_sync(0xffffffffu, mine.x, e);
+        const float p = __int_as_float(__shfl_sync(0xffffffffu, mine.y, e));
+        const bf16* vr = vbase + (size_t)j * DV;
+        if constexpr (PER == 8) {
+          const uint4 x = *reinterpret_cast<const uint4*>(vr);
+          acc[0] += p * bf16lo(x.x); acc[1] += p * bf16hi(x.x);
+          acc[2] += p * bf16lo(x.y); acc[3] += p * bf16hi(x.y);
+          acc[4] += p * bf16lo(x.z); acc[5] += p * bf16hi(x.z);
+          acc[6] += p * bf16lo(x.w); acc[7] += p * bf16hi(x.w);
+        } else if constexpr (PER == 4) {
+          const uint2 x = *reinterpret_cast<const uint2*>(vr);
+          acc[0] += p * bf16lo(x.x); acc[1] += p * bf16hi(x.x);
+          acc[2] += p * bf16lo(x.y); acc[3] += p * bf16hi(x.y);
+        } else {
+          const uint32_t x = *reinterpret_cast<const uint32_t*>(vr);
+          acc[0] += p * bf16lo(x); acc[1] += p * bf16hi(x);
+        }
+      }
+    }
+  }
+  bf16* o = P.out + flat * DV + lane * PER;
+#pragma unroll
+  for (int e = 0; e < PER; e += 2)
+    *reinterpret_cast<uint32_t*>(o + e) = pack_bf16(acc[e], acc[e + 1]);
+  if (lane == 0 && P.row_stat) P.row_stat[flat] = tau[flat];
 }
 
 }  // namespace nattn

@@ -1,0 +1,477 @@
+"""Benchmark of the fused attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload NAME] [--no-detail]
+
+A step is one forward of the workload for every normalizer the workload names
+(the Qwen3-8B-shaped prefill layer by default: B=2, Hq=32, Hkv=8 (GQA 4:1),
+T=4096, d=128, causal; softmax and softmax1).  Inputs are seeded synthetic
+bf16 tensors resident in HBM before timing starts; L2 is flushed (a 256 MiB
+write) before every timed step and the flush is outside the per-step CUDA
+events.  The headline value is useful TFLOP/s by the accounting rule of
+"Attention variants" (TensorCAD, "What the engine does today"):
+4 * T_eff * head_dim FLOPs per query row and head, halved when causal.
+
+Under torchrun each rank runs its own batch (independent problems, weak
+scaling, no data-path collective); the time is the max over ranks.
+
+--impl reference times the float64 CPU oracle on a bounded sample of the same
+workload on the host cores (the reference arm of this benchmark).
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+                  "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv",
+                 "-i", str(self.index), "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f.read().splitlines()[1:]:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm = float(parts[1].split()[0])
+                    smax = float(parts[2].split()[0])
+                except ValueError:
+                    continue
+                rows.append((sm, smax, parts[5:9]))
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, x in enumerate(r)
+                          if x.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------
+# native arm
+# --------------------------------------------------------------------------
+def kv_bytes_decode(x, w):
+    lens = x["seqlens"].long()
+    return int(lens.sum()) * w.Hkv * (w.d + w.dv) * 2 + \
+        2 * w.B * w.Hq * w.Tq * w.d * 2
+
+
+class Runner:
+    """Preallocated arguments and scratch for one workload on one device."""
+
+    def __init__(self, w, dev, seed_offset=0):
+        import torch
+        from alternative_normalizers_b200 import binding
+        from alternative_normalizers_b200.workloads import make_inputs
+        self.w = w
+        self.binding = binding
+        x = make_inputs(w, seed=w.seed + seed_offset)
+        self.host = x
+        self.x = {k: v.to(dev) for k, v in x.items()}
+        if w.paged:
+            self.out = torch.empty(w.B, w.Hq, w.Tq, w.dv, dtype=torch.bfloat16,
+                                   device=dev)
+            self.max_len = w.len_range[1]
+        else:
+            self.out = torch.empty(w.B, w.Hq, w.Tq, w.dv, dtype=torch.bfloat16,
+                                   device=dev)
+        self.stat = torch.empty(w.B, w.Hq, w.Tq, dtype=torch.float32, device=dev)
+        self.args = {}
+        self.ws = {}
+        stream = torch.cuda.current_stream(dev).cuda_stream
+        for n in w.normalizers:
+            a = self._args(n, self.x, self.out, self.stat, stream)
+            need = binding.nattn_workspace_size(a)
+            if need:
+                self.ws[n] = torch.empty(need, dtype=torch.uint8, device=dev)
+                a.workspace, a.workspace_bytes = self.ws[n].data_ptr(), need
+            self.args[n] = a
+
+    def _args(self, n, x, out, stat, stream):
+        w = self.w
+        if w.paged:
+            return self.binding.build_args(
+                x["q"], x["k_pool"], x["v_pool"], out, stat, None,
+                normalizer=n, causal=w.causal, window=w.window,
+                softcap=w.softcap, scale=w.scale, block_table=x["block_table"],
+                seqlens=x["seqlens"], page_size=w.page_size,
+                max_seqlen=self.max_len, stream=stream)
+        return self.binding.build_args(
+            x["q"], x["k"], x["v"], out, stat, None, normalizer=n,
+            causal=w.causal, window=w.window, softcap=w.softcap,
+            scale=w.scale, stream=stream)
+
+    def call(self, n):
+        rc = self.binding.nattn_fwd_ex(self.args[n])
+        if rc != 0:
+            raise RuntimeError(f"nattn_fwd_ex({n}) failed: {rc}")
+
+    def units(self):
+        """Useful FLOPs (prefill) or K/V bytes (decode) of one normalizer."""
+        if self.w.paged:
+            return kv_bytes_decode(self.host, self.w)
+        return self.w.useful_flops()
+
+
+LAUNCHES = {"softmax": 1, "softmax1": 1, "sparsemax": 3, "entmax15": 3}
+LAUNCHES_DECODE = {"softmax": 2, "softmax1": 2, "sparsemax": 4, "entmax15": 4}
+
+
+def time_runner(r, steps, warmup, flush):
+    """Per-normalizer average kernel time (ms) over `steps` timed steps, each
+    preceded by an L2 flush outside the events."""
+    import torch
+    for _ in range(warmup):
+        for n in r.w.normalizers:
+            r.call(n)
+    torch.cuda.synchronize()
+    ev = {n: [] for n in r.w.normalizers}
+    for _ in range(steps):
+        for n in r.w.normalizers:
+            flush.zero_()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(
+                enable_timing=True)
+            s.record()
+            r.call(n)
+            e.record()
+            ev[n].append((s, e))
+    torch.cuda.synchronize()
+    return {n: sum(s.elapsed_time(e) for s, e in v) / len(v)
+            for n, v in ev.items()}
+
+
+def e2e_measure(r, steps, dev):
+    """Same metric through the C ABI with host buffers: every step copies the
+    inputs from pinned host memory and reads the output and row statistics
+    back, all inside the timed region."""
+    import torch
+    host = {k: v.pin_memory() for k, v in r.host.items()}
+    dst = {k: torch.empty_like(v, device=dev) for k, v in r.host.items()}
+    out_h = torch.empty(r.out.shape, dtype=r.out.dtype).pin_memory()
+    stat_h = torch.empty(r.stat.shape, dtype=r.stat.dtype).pin_memory()
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    args = {n: r._args(n, dst, r.out, r.stat, stream) for n in r.w.normalizers}
+    for n, a in args.items():
+        if n in r.ws:
+            a.workspace = r.ws[n].data_ptr()
+            a.workspace_bytes = r.ws[n].numel()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_h.numel() * out_h.element_size() + stat_h.numel() * 4
+
+    def one():
+        for k in host:
+            dst[k].copy_(host[k], non_blocking=True)
+        for n in r.w.normalizers:
+            if r.binding.nattn_fwd_ex(args[n]) != 0:
+                raise RuntimeError("nattn_fwd_ex failed")
+            out_h.copy_(r.out, non_blocking=True)
+            stat_h.copy_(r.stat, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        one()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    nn = len(r.w.normalizers)
+    return ms, h2d, d2h * nn
+
+
+def cpu_baseline_prefill(w, x, budget_s=12.0):
+    """The float64 oracle on a bounded sample of query rows (head 0 of batch
+    0, evenly spaced rows), scaled to useful TFLOP/s."""
+    import numpy as np
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max(i.get("num_threads", 1) for i in threadpool_info()) \
+            if threadpool_info() else os.cpu_count()
+    except Exception:
+        cores = os.cpu_count()
+    q = x["q"][:1, :1]
+    g = 0
+    k = x["k"][:1, g:g + 1]
+    v = x["v"][:1, g:g + 1]
+    flops, secs, nrows, n_used = 0.0, 0.0, 0, 0
+    stride = max(1, w.Tq // 512)
+    rows_all = np.arange(w.Tq - 1, -1, -stride)
+    ok = oracle.allowed_matrix(w.Tq, w.Tk, w.causal, w.window)
+    t_start = time.perf_counter()
+    for n in w.normalizers:
+        for i0 in range(0, len(rows_all), 64):
+            sel = rows_all[i0:i0 + 64]
+            rows = np.stack([np.zeros_like(sel), np.zeros_like(sel), sel], 1)
+            t0 = time.perf_counter()
+            oracle.attention_rows(q, k, v, rows, w.scale, n, w.causal,
+                                  w.window, w.softcap)
+            secs += time.perf_counter() - t0
+            flops += float(ok[sel].sum()) * 4 * w.d
+            nrows += len(sel)
+            if time.perf_counter() - t_start > budget_s:
+                break
+        n_used += 1
+        if time.perf_counter() - t_start > budget_s:
+            break
+    return {"value": flops / secs / 1e12 if secs else None, "unit": "TFLOP/s",
+            "cores": cores, "kind": "oracle",
+            "sample": f"{nrows} query rows of head 0 (evenly spaced, latest "
+                      f"first) over {n_used} normalizer(s), float64 numpy, "
+                      f"{secs:.1f} s; FLOPs counted per visible key"}
+
+
+def main_native(args):
+    import torch
+    import torch.distributed as dist
+    from alternative_normalizers_b200 import binding
+    from alternative_normalizers_b200.workloads import WORKLOADS
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    binding.lib()
+
+    w = WORKLOADS[args.workload]
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    r = Runner(w, dev, seed_offset=rank)
+    for n in w.normalizers:  # warm-up, also the launch configuration checks
+        r.call(n)
+    torch.cuda.synchronize()
+    if binding.nattn_get_device_status() != 0:
+        raise RuntimeError("device status after warm-up")
+
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    per = time_runner(r, args.steps, args.warmup, flush)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms_step = sum(per.values())
+    if world > 1:
+        t = torch.tensor([ms_step], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+        dist.barrier()
+
+    units = r.units()
+    total_units = units * len(w.normalizers) * world
+    if w.paged:
+        value = total_units / (ms_step * 1e-3) / 1e9
+        unit, metric = "GB/s", "decode K/V GB/s (paged, split-KV)"
+    else:
+        value = total_units / (ms_step * 1e-3) / 1e12
+        unit, metric = "TFLOP/s", "fwd attention useful TFLOP/s (prefill)"
+
+    peaks, peak_src = load_peaks()
+    # dominant kernel: the prefill (or decode split) launch of one normalizer
+    dom = max(per, key=per.get)
+    if w.paged:
+        ach = units / (per[dom] * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peak,
+                "unit": "GB/s"}
+    else:
+        ach = units / (per[dom] * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": peak,
+                "unit": "TFLOP/s"}
+    roof["frac"] = round(ach / peak, 4)
+    roof["traffic"] = None
+    roof["kernel"] = f"{dom} launch"
+    roof["peak_source"] = (f"{peak_src} "
+                           f"{'hbm_gbs' if w.paged else 'bf16_tflops_sustained'}")
+
+    line = {
+        "metric": metric, "value": round(value, 2), "unit": unit,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded, see workloads.py)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
+                   "Tq": w.Tq, "Tk": w.Tk, "d": w.d, "dv": w.dv,
+                   "causal": w.causal, "window": w.window,
+                   "softcap": w.softcap,
+                   "normalizers": list(w.normalizers),
+                   "parallelism": f"independent batch per GPU x{world}",
+                   "l2": "flushed (256 MiB write) before every timed launch, "
+                         "outside the CUDA events"},
+        "per_normalizer_ms": {n: round(v, 4) for n, v in per.items()},
+        "per_normalizer_value": {
+            n: round(units / (v * 1e-3) / (1e9 if w.paged else 1e12), 2)
+            for n, v in per.items()},
+        "roofline": roof,
+        "clocks": clocks,
+        "gpu_launches": args.steps * sum(
+            (LAUNCHES_DECODE if w.paged else LAUNCHES)[n]
+            for n in w.normalizers),
+    }
+    if rank == 0:
+        e2e_ms, h2d, d2h = e2e_measure(r, max(3, args.steps // 4), dev)
+        e2e_val = units * len(w.normalizers) / (e2e_ms * 1e-3) / (
+            1e9 if w.paged else 1e12)
+        line["e2e"] = {"value": round(e2e_val, 3), "unit": unit,
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "ms_per_step": round(e2e_ms, 3)}
+        if world == 1 and not w.paged:
+            line["cpu_baseline"] = cpu_baseline_prefill(w, r.host)
+        if args.detail:
+            line["other_workloads"] = detail(args, dev, flush)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def detail(args, dev, flush):
+    """The other workload shapes, each normalizer timed like the headline."""
+    import torch
+    from alternative_normalizers_b200.workloads import WORKLOADS
+    res = {}
+    names = ["sparse_prefill_t1", "sparse_prefill_t4", "gemma2_9b_local",
+             "gemma2_9b_global", "paged_decode"]
+    for name in names:
+        w = WORKLOADS[name]
+        try:
+            r = Runner(w, dev)
+            per = time_runner(r, max(3, args.steps // 2), 2, flush)
+            u = r.units()
+            if w.paged:
+                vals = {n: round(u / (t * 1e-3) / 1e9, 1) for n, t in per.items()}
+                unit = "GB/s (dense-equivalent K/V bytes)"
+            else:
+                vals = {n: round(u / (t * 1e-3) / 1e12, 1) for n, t in per.items()}
+                unit = "useful TFLOP/s"
+            res[name] = {"unit": unit, "value": vals,
+                         "ms": {n: round(t, 4) for n, t in per.items()}}
+            del r
+            torch.cuda.empty_cache()
+        except Exception as exc:  # report, keep the headline line
+            res[name] = {"error": repr(exc)[:200]}
+    return res
+
+
+# --------------------------------------------------------------------------
+# reference arm: the float64 oracle on the host cores
+# --------------------------------------------------------------------------
+def main_reference(args):
+    from alternative_normalizers_b200.workloads import WORKLOADS, make_inputs
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    x = make_inputs(w)
+    budget = 4.0
+    vals = []
+    cb = None
+    for _ in range(args.warmup):
+        cpu_baseline_prefill(w, x, budget_s=1.0)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        cb = cpu_baseline_prefill(w, x, budget_s=budget)
+        vals.append(cb["value"])
+    wall = time.perf_counter() - t0
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": "fwd attention useful TFLOP/s (prefill)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(wall / max(1, args.steps) * 1e3, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded, see workloads.py)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
+                   "Tq": w.Tq, "Tk": w.Tk, "d": w.d, "causal": w.causal,
+                   "normalizers": list(w.normalizers)},
+        "cpu_baseline": dict(cb, value=value),
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="native", choices=["native", "reference"])
+    p.add_argument("--workload", default="qwen3_8b_prefill")
+    p.add_argument("--no-detail", dest="detail", action="store_false")
+    args = p.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        main_reference(args)
+    else:
+        main_native(args)
+
+
+if __name__ == "__main__":
+    main()
