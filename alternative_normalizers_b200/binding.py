@@ -79,6 +79,8 @@ def lib():
         L.nattn_strerror.restype = ctypes.c_char_p
         L.nattn_version.argtypes = []
         L.nattn_version.restype = ctypes.c_int
+        L.nattn_decode_noalloc.argtypes = [P]
+        L.nattn_decode_noalloc.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -114,6 +116,12 @@ def nattn_strerror(code):
 
 def nattn_version():
     return lib().nattn_version()
+
+
+def nattn_decode_noalloc(args: NattnArgs):
+    """Paged softmax/softmax1 decode with the library's fixed scratch array:
+    no workspace, no allocation (``args.workspace`` is ignored)."""
+    return lib().nattn_decode_noalloc(ctypes.byref(args))
 
 
 # --------------------------------------------------------------------------

@@ -7,6 +7,7 @@
 //   dense, head dims 64/128/256 (d == dv)-> tcgen05 prefill kernels
 //   anything else that validates         -> row-wise kernel
 #include <math.h>
+#include <mutex>
 #include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
@@ -431,6 +432,75 @@ int run(const nattn_args* a) {
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Allocation-free paged decode: split partials in a fixed device array
+// ---------------------------------------------------------------------------
+// The array is this file's own; host code only ever sees a stand-in for its
+// name, so the device address is looked up once per device and cached.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NATTN_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kNoAllocDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kNoAllocDevices] = {};
+
+// Device address of the scratch array on the current device (first call per
+// device does the lookup with that device current).
+int noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocDevices)
+    return NATTN_ECUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return NATTN_ECUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return NATTN_OK;
+}
+
+int decode_noalloc(const nattn_args* a) {
+  int rc = validate(a);
+  if (rc != NATTN_OK) return rc;
+  if (a->B == 0 || a->Hq == 0 || a->Tq == 0) return NATTN_OK;
+  if (!is_paged(a)) return NATTN_EUNSUPPORTED;
+  if (a->normalizer != NATTN_SOFTMAX && a->normalizer != NATTN_SOFTMAX1)
+    return NATTN_EUNSUPPORTED;
+  Plan pl = make_plan(a);
+  if (pl.path != PATH_DECODE) return NATTN_EUNSUPPORTED;
+  // choose the split count so that the partials fit the array
+  const size_t rows_per_split = (size_t)a->B * a->Hkv * pl.R;
+  const size_t per_split = up256(rows_per_split * a->dv * 4) + up256(rows_per_split * 2 * 4);
+  const int fit = (int)(NATTN_NOALLOC_SCRATCH_BYTES / per_split);
+  if (fit < 1) return NATTN_ETOOLARGE;
+  const int maxp = (a->Tk + a->page_size - 1) / a->page_size;
+  if (pl.nsplit > fit) {
+    pl.pps = (maxp + fit - 1) / fit;
+    pl.nsplit = (maxp + pl.pps - 1) / pl.pps;
+  }
+  const size_t parts = rows_per_split * pl.nsplit;
+  pl.off_opart = 0;
+  pl.off_ml = up256(parts * a->dv * 4);
+  pl.total = pl.off_ml + up256(parts * 2 * 4);
+  if (pl.total > NATTN_NOALLOC_SCRATCH_BYTES) return NATTN_ETOOLARGE;
+  void* base = nullptr;
+  rc = noalloc_scratch(&base);
+  if (rc != NATTN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(a->stream);
+  const Problem P = to_problem(a);
+  uint8_t* ws = static_cast<uint8_t*>(base);
+  if (a->page_size == 32) {
+    if (a->d == 64) return launch_decode<64, 32>(a, P, pl, ws, st);
+    if (a->d == 128) return launch_decode<128, 32>(a, P, pl, ws, st);
+    return launch_decode<256, 32>(a, P, pl, ws, st);
+  }
+  if (a->d == 64) return launch_decode<64, 64>(a, P, pl, ws, st);
+  if (a->d == 128) return launch_decode<128, 64>(a, P, pl, ws, st);
+  return launch_decode<256, 64>(a, P, pl, ws, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -514,5 +584,9 @@ __attribute__((visibility("default"))) const char* nattn_strerror(int code) {
 }
 
 __attribute__((visibility("default"))) int nattn_version(void) { return kVersion; }
+
+__attribute__((visibility("default"))) int nattn_decode_noalloc(const nattn_args* a) {
+  return decode_noalloc(a);
+}
 
 }  // extern "C"

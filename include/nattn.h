@@ -167,6 +167,40 @@ int nattn_get_device_status(void* stream);
 /* Static description of an error code. */
 const char* nattn_strerror(int code);
 
+/*
+ * Paged decode that allocates nothing (no paper counterpart; a deployment
+ * convenience of this library).
+ *
+ * Some callers cannot allocate device memory at the point where they run
+ * attention: a serving loop whose memory is owned by another allocator, a
+ * plugin that is handed pointers but no allocator, or a latency-critical
+ * decode step that must not risk the implicit synchronisation of
+ * cudaMalloc.  This entry point takes the same argument block as
+ * nattn_fwd_ex in paged mode but ignores `workspace`: its split-KV partial
+ * results live in a fixed device array inside the library, of
+ * NATTN_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the library
+ * holds until the process exits.
+ *
+ *   - Supported: paged mode, NATTN_SOFTMAX or NATTN_SOFTMAX1, d == dv in
+ *     {64, 128, 256}, page_size 32 or 64, (Hq / Hkv) * Tq <= 16.  Anything
+ *     else returns NATTN_EUNSUPPORTED.
+ *   - The split count is chosen so the partials fit the array; a batch whose
+ *     partials do not fit even with one split per sequence
+ *     (B * Hkv * (Hq / Hkv) * Tq * (dv + 2) * 4 bytes > the array) returns
+ *     NATTN_ETOOLARGE and launches nothing.
+ *   - The first call on a device looks up that device's address of the
+ *     array (cudaGetSymbolAddress, with the device current); make that first
+ *     call outside any stream capture.
+ *   - Every call shares the one array and leaves its contents behind.  The
+ *     kernels overwrite every partial they later read, so nothing has to
+ *     start at zero, but calls that overlap on the GPU (other streams, other
+ *     host threads) race on the array: order them on one stream.
+ *   - Calls no cudaMalloc, cudaFree or other allocating routine.
+ * Returns NATTN_OK or a negative error code; asynchronous on a->stream.
+ */
+#define NATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
+int nattn_decode_noalloc(const nattn_args* a);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 int nattn_version(void);
 
