@@ -133,6 +133,28 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+// Bounded wait that polls with a short sleep between polls instead of asking
+// to be suspended: for waits whose reaction time is on the critical path
+// (the MMA issuer, the normalizer warps), while leaving the issue slots of
+// the sub-partition to the warps that share it.
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity,
+                                               volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(20);
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (abort != nullptr && *abort) return false;
+      if (globaltimer() - t0 > NATTN_WAIT_NS) {
+        set_status(NATTN_ETIMEOUT);
+        if (abort != nullptr) *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // TMA (tensor and plain bulk copies, global -> shared, no multicast)
 // ---------------------------------------------------------------------------

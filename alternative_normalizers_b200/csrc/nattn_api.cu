@@ -296,10 +296,12 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
     A.sup_count = nullptr;
     A.sup_list = nullptr;
     A.sup_cap = 0;
-    using LY = TcLayout<D, D, BN, KST, VST, TC_ONLINE>;
-    auto k = prefill_tc_kernel<D, D, BN, KST, VST, TC_ONLINE>;
+    // split each S row between two warps where TMEM holds two O halves
+    constexpr int NH = (2 * BN + 2 * D <= 512) ? 2 : 1;
+    using LY = TcLayout<D, D, BN, KST, VST, TC_ONLINE, NH>;
+    auto k = prefill_tc_kernel<D, D, BN, KST, VST, TC_ONLINE, NH>;
     if (allow_smem(k, LY::ALLOC) != cudaSuccess) return NATTN_ECUDA;
-    k<<<grid, TC_THREADS, LY::ALLOC, st>>>(mq, mk, mv, A);
+    k<<<grid, LY::THREADS, LY::ALLOC, st>>>(mq, mk, mv, A);
     return check_launch();
   }
   const float us = (a->normalizer == NATTN_ENTMAX15) ? 0.5f : 1.0f;
@@ -316,14 +318,14 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
     using LY = TcLayout<D, D, BN, 2, 1, TC_TAU>;
     auto k = prefill_tc_kernel<D, D, BN, 2, 1, TC_TAU>;
     if (allow_smem(k, LY::ALLOC) != cudaSuccess) return NATTN_ECUDA;
-    k<<<grid, TC_THREADS, LY::ALLOC, st>>>(mq, mk, mv, A);
+    k<<<grid, LY::THREADS, LY::ALLOC, st>>>(mq, mk, mv, A);
     if (check_launch() != NATTN_OK) return NATTN_ECUDA;
   }
   if (pl.tc_apply) {
     using LY = TcLayout<D, D, BN, KST, VST, TC_APPLY>;
     auto k = prefill_tc_kernel<D, D, BN, KST, VST, TC_APPLY>;
     if (allow_smem(k, LY::ALLOC) != cudaSuccess) return NATTN_ECUDA;
-    k<<<grid, TC_THREADS, LY::ALLOC, st>>>(mq, mk, mv, A);
+    k<<<grid, LY::THREADS, LY::ALLOC, st>>>(mq, mk, mv, A);
     if (check_launch() != NATTN_OK) return NATTN_ECUDA;
   } else {
     const size_t rows = (size_t)a->B * a->Hq * a->Tq;
@@ -341,7 +343,8 @@ template <int D, int PS, int MODE>
 int launch_decode_mode(const nattn_args* a, const DecodeArgs& A, const CUtensorMap& mk,
                        const CUtensorMap& mv, cudaStream_t st) {
   using L1 = DecodeSmem<D, D, PS, 2, MODE>;
-  constexpr int NS = (L1::STAGE * 4 <= 128 * 1024) ? 4 : (L1::STAGE * 3 <= 200 * 1024 ? 3 : 2);
+  // about 100 KB of stages: two CTAs per SM for K+V pages, three for K or V
+  constexpr int NS = (L1::STAGE * 4 <= 100 * 1024) ? 4 : (L1::STAGE * 3 <= 100 * 1024 ? 3 : 2);
   using L = DecodeSmem<D, D, PS, NS, MODE>;
   const int bytes = L::BYTES_NOLIST + 2 * A.pps * 4 + 1024;
   dim3 grid(A.nsplit, a->Hkv, a->B);

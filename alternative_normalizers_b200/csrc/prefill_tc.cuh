@@ -50,7 +50,7 @@ constexpr int TC_BM = 128;
 // candidate buffer entries per row in the threshold pass (value + key index)
 template <int D>
 struct TauCap {
-  static constexpr int value = (D >= 256) ? 64 : 128;
+  static constexpr int value = (D >= 256) ? 88 : 112;
 };
 
 struct TcArgs {
@@ -65,8 +65,16 @@ struct TcArgs {
   int sup_cap;
 };
 
-template <int D, int DV, int BN, int KST, int VST, int MODE>
+// NH = 2 splits every S row between two warps (columns [0, BN/2) and
+// [BN/2, BN)); each half keeps its own running maximum, denominator and O
+// accumulator in TMEM, and the halves are merged once in the epilogue.  Two
+// normalizer warps per SM sub-partition hide each other's latency and each
+// thread holds half a row in registers.
+template <int D, int DV, int BN, int KST, int VST, int MODE, int NH = 1>
 struct TcLayout {
+  static_assert(NH == 1 || MODE == TC_ONLINE, "row split is for the online mode");
+  static constexpr int NWN = 4 * NH;                 // normalizer warps
+  static constexpr int THREADS = (NWN + 2) * 32;     // + TMA warp + MMA warp
   static constexpr int QBYTES = D * TC_BM * 2;
   static constexpr int KBYTES = D * BN * 2;
   static constexpr int VBYTES = (MODE == TC_TAU) ? 0 : DV * BN * 2;
@@ -75,18 +83,21 @@ struct TcLayout {
   static constexpr int OFF_V = OFF_K + KST * KBYTES;
   static constexpr int OFF_BUF = OFF_V + VST * VBYTES;
   static constexpr int CAP = TauCap<D>::value;
-  static constexpr int BUFBYTES = (MODE == TC_TAU) ? 2 * CAP * TC_BM * 4 : 0;
-  static constexpr int OFF_IDX = OFF_BUF + CAP * TC_BM * 4;
+  static constexpr int CAP_STRIDE = CAP + 1;  // int2 entries per row
+  static constexpr int BUFBYTES = (MODE == TC_TAU) ? CAP_STRIDE * TC_BM * 8 : 0;
   static constexpr int OFF_BAR = OFF_BUF + BUFBYTES;
   static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 2 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  // epilogue (m, l) exchange between row halves: reuses the Q tile, which
+  // every product has finished reading once the last PV has completed
+  static constexpr int OFF_XCH = OFF_Q;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
   // TMEM columns: S double buffer, then O
   static constexpr int TM_S0 = 0;
   static constexpr int TM_S1 = BN;
   static constexpr int TM_O = 2 * BN;
-  static constexpr int TM_COLS_USED = (MODE == TC_TAU) ? 2 * BN : 2 * BN + DV;
+  static constexpr int TM_COLS_USED = (MODE == TC_TAU) ? 2 * BN : 2 * BN + NH * DV;
   static constexpr int TM_COLS = TM_COLS_USED <= 32    ? 32
                                  : TM_COLS_USED <= 64  ? 64
                                  : TM_COLS_USED <= 128 ? 128
@@ -102,26 +113,54 @@ __device__ __forceinline__ float tc_z(float s, const TcArgs& A) {
   return s * A.zscale;
 }
 
-// Per-thread exact threshold over the candidate buffer (values in threshold
-// units u).  Same method as the block-level solver of the row-wise kernel:
-// Newton from the left on g(t) = sum relu(u - t)^k, accepting the closed-form
-// threshold of {u > t} once it satisfies the optimality conditions.
-// `t0` is a lower bound of tau in shifted units (u - m).  With `newton_only`
-// it returns after `iters` Newton steps (a valid lower bound, for pruning).
-__device__ __noinline__ float thread_tau(const float* buf, int n, float m, bool entmax,
-                                            float t0, int iters, bool newton_only) {
+// Exact threshold of one row's candidate buffer, computed by the whole warp
+// (every lane holds up to four entries of that row in registers).  Values are
+// in threshold units u; `m` is the row maximum, `t0` a lower bound of tau in
+// shifted units (u - m).
+//
+// Newton's method from the left on g(t) = sum relu(u - t)^k - 1 (k = 1 for
+// sparsemax, 2 for 1.5-entmax), which is convex and decreasing, so every
+// iterate stays at or below the root and {u > t} always contains the
+// support.  At each iterate the closed-form threshold of that set is tried
+// first and accepted once it satisfies the optimality conditions (all members
+// above it, everything else at or below it); for sparsemax this is Michelot's
+// projection algorithm.
+struct RowEntries {
+  int2 e[4];  // (key index, value bits); value -inf marks an empty slot
+};
+
+__device__ __forceinline__ RowEntries warp_load_row(const int2* row, int n) {
+  const int lane = threadIdx.x & 31;
+  RowEntries r;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int k = lane + 32 * i;
+    r.e[i] = (k < n) ? row[k] : make_int2(0, __float_as_int(-INFINITY));
+  }
+  return r;
+}
+
+__device__ __forceinline__ float warp_row_tau(const RowEntries& r, float m, bool entmax,
+                                              float t0) {
+  float w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) w[i] = __int_as_float(r.e[i].y) - m;
   float t = fmaxf(t0, -1.f);
-  for (int it = 0; it < iters; ++it) {
+  for (int it = 0; it < 64; ++it) {
     float cnt = 0.f, s1 = 0.f, s2 = 0.f, wmin = INFINITY;
-    for (int k = 0; k < n; ++k) {
-      const float w = buf[k * TC_BM] - m;
-      if (w > t) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (w[i] > t) {
         cnt += 1.f;
-        s1 += w;
-        s2 += w * w;
-        wmin = fminf(wmin, w);
+        s1 += w[i];
+        s2 += w[i] * w[i];
+        wmin = fminf(wmin, w[i]);
       }
     }
+    cnt = warp_sum(cnt);
+    s1 = warp_sum(s1);
+    s2 = warp_sum(s2);
+    wmin = warp_min(wmin);
     float ts, tn;
     bool valid = true;
     if (!entmax) {
@@ -136,19 +175,38 @@ __device__ __noinline__ float thread_tau(const float* buf, int n, float m, bool 
       const float gp = 2.f * (s1 - t * cnt);
       tn = t + (g - 1.f) / gp;
     }
-    if (!newton_only && valid && ts >= t && wmin > ts) return ts + m;
+    if (valid && ts >= t && wmin > ts) return ts + m;
     if (!(tn > t)) break;
     t = tn;
   }
   return t + m;
 }
 
-template <int D, int DV, int BN, int KST, int VST, int MODE>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+// Keep the entries above `lb`, compacted to the front of `row`; returns the
+// new count.  Reads happened in warp_load_row, so writing in place is safe.
+__device__ __forceinline__ int warp_compact_row(const RowEntries& r, int2* row, float lb) {
+  const int lane = threadIdx.x & 31;
+  const unsigned below = (1u << lane) - 1u;
+  int base = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const bool keep = __int_as_float(r.e[i].y) > lb;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (keep) row[base + __popc(bal & below)] = r.e[i];
+    base += __popc(bal);
+  }
+  __syncwarp();
+  return base;
+}
+
+template <int D, int DV, int BN, int KST, int VST, int MODE, int NH = 1>
+__global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                       const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, TcArgs A) {
-  using LY = TcLayout<D, DV, BN, KST, VST, MODE>;
+  using LY = TcLayout<D, DV, BN, KST, VST, MODE, NH>;
+  constexpr int NWN = LY::NWN;
+  constexpr int NC = BN / NH;  // S columns per normalizer thread
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -196,13 +254,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar_sfull(s), 1);
-      mbar_init(bar_pfull(s), 4);
+      mbar_init(bar_pfull(s), NWN);
     }
     mbar_init(bar_pv, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == NWN + 1) {
     tmem_alloc(smem_addr(&misc[0]), LY::TM_COLS);
     tmem_relinquish();
   }
@@ -211,7 +269,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = misc[0];
 
-  if (warp == 4) {
+  if (warp == NWN) {
     // ======================= TMA producer ===================================
     if (lane == 0 && nblk > 0) {
       tma_prefetch_desc(&tmq);
@@ -245,25 +303,26 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == NWN + 1) {
     // ======================= MMA issuer =====================================
     if (lane == 0 && nblk > 0) {
       constexpr uint32_t IDESC_S = idesc_bf16(TC_BM, BN, 0, 0);
       constexpr uint32_t IDESC_O = idesc_bf16(TC_BM, DV, 0, 1);
       const uint32_t qbase = smem_addr(smem + LY::OFF_Q);
-      bool ok = mbar_wait(bar_q, 0, abort_flag);
+      bool ok = mbar_wait_spin(bar_q, 0, abort_flag);
       tc_fence_after();
       for (int j = 0; ok && j <= nblk; ++j) {
         if (j < nblk) {
           const int sb = j & 1, ks = j % KST;
-          if (!mbar_wait(bar_kfull(ks), (j / KST) & 1, abort_flag)) break;
-          if (j >= 2) {
-            // S buffer sb is free once P_{j-2} has been consumed
-            if constexpr (MODE == TC_TAU) {
-              if (!mbar_wait(bar_pfull(sb), ((j - 2) / 2) & 1, abort_flag)) break;
-            } else {
-              if (!mbar_wait(bar_pv, (j - 2) & 1, abort_flag)) break;
-            }
+          if (!mbar_wait_spin(bar_kfull(ks), (j / KST) & 1, abort_flag)) break;
+          // S buffer sb held P_{j-2}.  With a PV product that reads it, that
+          // product was issued by this thread before this QK and tcgen05.mma
+          // operations from one thread execute in issue order, so no wait is
+          // needed; without one (threshold pass) the normalizer warps must be
+          // done reading S_{j-2}.
+          if constexpr (MODE == TC_TAU) {
+            if (j >= 2 && !mbar_wait_spin(bar_pfull(sb), ((j - 2) / 2) & 1, abort_flag))
+              break;
           }
           tc_fence_after();
           const uint32_t kbase = smem_addr(smem + LY::OFF_K + ks * LY::KBYTES);
@@ -282,18 +341,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if constexpr (MODE != TC_TAU) {
           if (j >= 1) {
             const int jp = j - 1, sbp = jp & 1, vs = jp % VST;
-            if (!mbar_wait(bar_pfull(sbp), (jp / 2) & 1, abort_flag)) break;
-            if (!mbar_wait(bar_vfull(vs), (jp / VST) & 1, abort_flag)) break;
+            if (!mbar_wait_spin(bar_pfull(sbp), (jp / 2) & 1, abort_flag)) break;
+            if (!mbar_wait_spin(bar_vfull(vs), (jp / VST) & 1, abort_flag)) break;
             tc_fence_after();
             const uint32_t vbase = smem_addr(smem + LY::OFF_V + vs * LY::VBYTES);
             const uint32_t pt = tmem + (sbp ? LY::TM_S1 : LY::TM_S0);
 #pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk) {
-              // V block is [BN keys][DV] in 64-column boxes: MN-major B
-              // operand, LBO = box stride, SBO = 8 key rows.
-              const uint64_t bd = sdesc_sw128(vbase + kk * 16 * 128, BN * 128, 1024);
-              umma_ts(tmem + LY::TM_O, pt + kk * 8, bd, IDESC_O,
-                      (jp > 0 || kk > 0) ? 1u : 0u);
+            for (int hh = 0; hh < NH; ++hh) {
+              // half hh: its packed P sits at the start of its own S columns,
+              // its keys are V rows [hh * NC, (hh + 1) * NC)
+#pragma unroll
+              for (int kk = 0; kk < NC / 16; ++kk) {
+                // V block is [BN keys][DV] in 64-column boxes: MN-major B
+                // operand, LBO = box stride, SBO = 8 key rows.
+                const uint64_t bd =
+                    sdesc_sw128(vbase + (hh * NC + kk * 16) * 128, BN * 128, 1024);
+                umma_ts(tmem + LY::TM_O + hh * DV, pt + hh * NC + kk * 8, bd, IDESC_O,
+                        (jp > 0 || kk > 0) ? 1u : 0u);
+              }
             }
             umma_commit(bar_vempty(vs));
             umma_commit(bar_pv);
@@ -302,14 +367,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
     }
   } else {
-    // ======================= normalizer warps (0-3) ========================
-    const int row = warp * 32 + lane;
+    // ======================= normalizer warps ==============================
+    const int quarter = warp & 3;        // TMEM lane quarter = query rows
+    const int half = warp >> 2;          // which columns of the S row
+    const int cbase = half * NC;
+    const int row = quarter * 32 + lane;
     const int qi = q0 + row;
     const bool row_ok = qi < P.Tq;
     RowRange rr = row_range(P, qi, P.Tk);
     if (!row_ok) rr = RowRange{1, 0};
     if (rr.hi > P.Tk - 1) rr.hi = P.Tk - 1;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const size_t flat = ((size_t)bh * P.Tq + qi);
     // fast path: no soft-cap and a positive scale, so max(z) = scale * max(s)
     // and exp2(z - m) is one FFMA + EX2 per score
@@ -318,14 +386,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
     float m_run, l_run = 0.f, tau = 0.f;
     // TAU state
-    float* buf = reinterpret_cast<float*>(smem + LY::OFF_BUF) + row;
-    int* bidx = reinterpret_cast<int*>(smem + LY::OFF_IDX) + row;
+    int2* tbuf = reinterpret_cast<int2*>(smem + LY::OFF_BUF) +
+                 (size_t)(quarter * 32) * LY::CAP_STRIDE;  // this warp's 32 rows
+    int2* mybuf = tbuf + lane * LY::CAP_STRIDE;
     int nbuf = 0;
     bool ovf = false;
     float lb = -INFINITY;  // lower bound of tau (threshold units)
     if constexpr (MODE == TC_ONLINE) {
-      m_run = (P.norm == NATTN_SOFTMAX1) ? 0.f : -INFINITY;
-      l_run = (P.norm == NATTN_SOFTMAX1) ? 1.f : 0.f;
+      // the softmax1 sink belongs to exactly one half of the row
+      const bool sink = P.norm == NATTN_SOFTMAX1 && half == 0;
+      m_run = sink ? 0.f : -INFINITY;
+      l_run = sink ? 1.f : 0.f;
     } else {
       m_run = -INFINITY;
     }
@@ -335,26 +406,26 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
     for (int j = 0; j < nblk; ++j) {
       const int sb = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_sfull(sb), (j / 2) & 1, abort_flag))) {
+      if (!__all_sync(0xffffffffu, mbar_wait_spin(bar_sfull(sb), (j / 2) & 1, abort_flag))) {
         alive = false;
         break;
       }
       tc_fence_after();
-      const int j0 = (kb0 + j) * BN;
-      const bool edge = !(rr.lo <= j0 && rr.hi >= j0 + BN - 1);
+      const int j0 = (kb0 + j) * BN + cbase;  // first key of this thread's columns
+      const bool edge = !(rr.lo <= j0 && rr.hi >= j0 + NC - 1);
       // visible keys of this row inside the block: [kl, kl + span]
       int kl = rr.lo - j0;
       unsigned span = (unsigned)(rr.hi - rr.lo);
       if (rr.hi < rr.lo) {
-        kl = BN;
+        kl = NC;
         span = 0;
       }
-      const uint32_t saddr = lane_base + (sb ? LY::TM_S1 : LY::TM_S0);
+      const uint32_t saddr = lane_base + (sb ? LY::TM_S1 : LY::TM_S0) + cbase;
 
-      // the whole S row of this block, one TMEM round trip
-      uint32_t r[BN];
+      // this thread's part of the S row, one TMEM round trip
+      uint32_t r[NC];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c)
+      for (int c = 0; c < NC / 32; ++c)
         tmem_ld32(saddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
       tmem_ld_wait();
 
@@ -362,18 +433,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       // masked entries become -inf
       if (!fast) {
 #pragma unroll
-        for (int k = 0; k < BN; ++k) r[k] = __float_as_uint(tc_z(__uint_as_float(r[k]), A));
+        for (int k = 0; k < NC; ++k) r[k] = __float_as_uint(tc_z(__uint_as_float(r[k]), A));
       }
       if (edge) {
 #pragma unroll
-        for (int k = 0; k < BN; ++k)
+        for (int k = 0; k < NC; ++k)
           if ((unsigned)(k - kl) > span) r[k] = __float_as_uint(-INFINITY);
       }
 
       if constexpr (MODE == TC_ONLINE) {
         float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-        for (int k = 0; k < BN; k += 4) {
+        for (int k = 0; k < NC; k += 4) {
           mx0 = fmaxf(mx0, __uint_as_float(r[k]));
           mx1 = fmaxf(mx1, __uint_as_float(r[k + 1]));
           mx2 = fmaxf(mx2, __uint_as_float(r[k + 2]));
@@ -389,7 +460,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const float fa = fast ? zs : 1.f;  // p = exp2(x * fa - msafe)
         float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int c = 0; c < BN / 64; ++c) {  // 64 scores -> 32 packed columns
+        for (int c = 0; c < NC / 64; ++c) {  // 64 scores -> 32 packed columns
           uint32_t pk[32];
 #pragma unroll
           for (int k = 0; k < 64; k += 2) {
@@ -411,7 +482,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t oaddr = lane_base + LY::TM_O;
+          const uint32_t oaddr = lane_base + LY::TM_O + half * DV;
 #pragma unroll 1
           for (int c = 0; c < DV / 32; ++c) {
             uint32_t o[32];
@@ -428,7 +499,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // p = relu(z - tau) or relu(z/2 - tau)^2 as bf16 P
         const float fa = fast ? zs : 1.f;
 #pragma unroll
-        for (int c = 0; c < BN / 64; ++c) {
+        for (int c = 0; c < NC / 64; ++c) {
           uint32_t pk[32];
 #pragma unroll
           for (int k = 0; k < 64; k += 2) {
@@ -445,7 +516,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         tmem_st_wait();
       } else {  // TC_TAU
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < NC / 32; ++c) {
           float cmax = -INFINITY;
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
@@ -454,27 +525,33 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
           m_run = fmaxf(m_run, cmax);
           lb = fmaxf(lb, m_run - 1.f);  // tau >= max - 1
-          if (cmax > lb && !ovf) {
-            if (nbuf + 32 > LY::CAP) {
-              // raise the lower bound with a few Newton steps, then compact
-              lb = thread_tau(buf, nbuf, m_run, entmax, lb - m_run, 4, true);
-              int w = 0;
-              for (int k = 0; k < nbuf; ++k) {
-                const float x = buf[k * TC_BM];
-                if (x > lb) {
-                  bidx[w * TC_BM] = bidx[k * TC_BM];
-                  buf[(w++) * TC_BM] = x;
-                }
-              }
-              nbuf = w;
+          const bool want = cmax > lb && !ovf;
+          // rows whose buffer could overflow on this chunk: raise their
+          // bound to the exact threshold of the keys seen so far (adding keys
+          // only raises tau), then compact; the whole warp works on one row
+          unsigned need = __ballot_sync(0xffffffffu, want && nbuf + 32 > LY::CAP);
+          while (need) {
+            const int rr_ = __ffs(need) - 1;
+            need &= need - 1;
+            const int n_r = __shfl_sync(0xffffffffu, nbuf, rr_);
+            const float m_r = __shfl_sync(0xffffffffu, m_run, rr_);
+            const float lb_r = __shfl_sync(0xffffffffu, lb, rr_);
+            int2* rowp = tbuf + rr_ * LY::CAP_STRIDE;
+            const RowEntries ent = warp_load_row(rowp, n_r);
+            const float nlb = warp_row_tau(ent, m_r, entmax, lb_r - m_r);
+            const int kept = warp_compact_row(ent, rowp, nlb);
+            if (lane == rr_) {
+              lb = nlb;
+              nbuf = kept;
             }
+          }
+          if (want && cmax > lb) {
 #pragma unroll
             for (int k = 0; k < 32; ++k) {
               const float u = __uint_as_float(r[c * 32 + k]);
               if (u > lb) {
                 if (nbuf < LY::CAP) {
-                  buf[nbuf * TC_BM] = u;
-                  bidx[nbuf * TC_BM] = j0 + c * 32 + k;
+                  mybuf[nbuf] = make_int2(j0 + c * 32 + k, __float_as_int(u));
                   ++nbuf;
                 } else {
                   ovf = true;
@@ -491,71 +568,115 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
     // ---- epilogue ----------------------------------------------------------
     if constexpr (MODE == TC_TAU) {
-      if (row_ok) {
+      // exact tau and the support list of every row, one row at a time with
+      // the whole warp
+      __syncwarp();
+      for (int rr_ = 0; rr_ < 32; ++rr_) {
+        const int qr = q0 + warp * 32 + rr_;
+        if (qr >= P.Tq) break;
+        const size_t fr = (size_t)bh * P.Tq + qr;
+        const int n_r = __shfl_sync(0xffffffffu, nbuf, rr_);
+        const float m_r = __shfl_sync(0xffffffffu, m_run, rr_);
+        const float lb_r = __shfl_sync(0xffffffffu, lb, rr_);
+        const bool ovf_r = __shfl_sync(0xffffffffu, (int)ovf, rr_) != 0;
         float t = INFINITY;
         int nsup = 0;
-        if (ovf) {
-          const int slot = atomicAdd(A.ovf_count, 1);
-          A.ovf_rows[slot] = (int)flat;
-        } else if (m_run != -INFINITY) {
-          t = thread_tau(buf, nbuf, m_run, entmax, lb - m_run, 64, false);
-          // the support and its weights, for the gather pass
-          int2* dst = A.sup_list + flat * (size_t)A.sup_cap;
-          for (int k = 0; k < nbuf; ++k) {
-            const float x = buf[k * TC_BM] - t;
-            if (x > 0.f) {
-              const float w = entmax ? x * x : x;
-              dst[nsup++] = make_int2(bidx[k * TC_BM], __float_as_int(w));
-            }
+        if (ovf_r) {
+          if (lane == 0) {
+            const int slot = atomicAdd(A.ovf_count, 1);
+            A.ovf_rows[slot] = (int)fr;
+          }
+        } else if (m_r != -INFINITY) {
+          const RowEntries ent = warp_load_row(tbuf + rr_ * LY::CAP_STRIDE, n_r);
+          t = warp_row_tau(ent, m_r, entmax, lb_r - m_r);
+          int2* dst = A.sup_list + fr * (size_t)A.sup_cap;
+          const unsigned below = (1u << lane) - 1u;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float x = __int_as_float(ent.e[i].y) - t;
+            const bool in = x > 0.f;
+            const unsigned bal = __ballot_sync(0xffffffffu, in);
+            if (in)
+              dst[nsup + __popc(bal & below)] =
+                  make_int2(ent.e[i].x, __float_as_int(entmax ? x * x : x));
+            nsup += __popc(bal);
           }
         }
-        A.tau[flat] = t;
-        A.sup_count[flat] = nsup;
+        if (lane == 0) {
+          A.tau[fr] = t;
+          A.sup_count[fr] = nsup;
+        }
       }
     } else {
       const bool have_o =
           __all_sync(0xffffffffu, alive && nblk > 0 &&
                                       mbar_wait(bar_pv, (nblk - 1) & 1, abort_flag));
       tc_fence_after();
-      float inv = 1.f, stat = tau;
+      // combine the halves: scale factors ca (half 0) and cb (half 1)
+      float ca = 1.f, cb = 0.f, stat = tau;
       if constexpr (MODE == TC_ONLINE) {
-        inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
-        const float msafe = (m_run == -INFINITY) ? 0.f : m_run;
-        stat = (l_run > 0.f) ? (msafe + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+        float m0 = m_run, l0 = l_run, m1 = -INFINITY, l1 = 0.f;
+        if constexpr (NH > 1) {
+          float2* xch = reinterpret_cast<float2*>(smem + LY::OFF_XCH);
+          xch[half * TC_BM + row] = make_float2(m_run, l_run);
+          asm volatile("bar.sync 1, %0;" ::"r"(NWN * 32) : "memory");
+          const float2 a0 = xch[row], a1 = xch[TC_BM + row];
+          m0 = a0.x;
+          l0 = a0.y;
+          m1 = a1.x;
+          l1 = a1.y;
+        }
+        const float M = fmaxf(m0, m1);
+        const float msafe = (M == -INFINITY) ? 0.f : M;
+        const float e0 = fast_exp2(m0 - msafe), e1 = fast_exp2(m1 - msafe);
+        const float l = l0 * e0 + l1 * e1;
+        const float inv = (l > 0.f) ? 1.f / l : 0.f;
+        ca = e0 * inv;
+        cb = e1 * inv;
+        stat = (l > 0.f) ? (msafe + log2f(l)) * 0.6931471805599453f : -INFINITY;
       }
-      bf16* orow = P.out + flat * DV;
-      const uint32_t oaddr = lane_base + LY::TM_O;
+      // this thread writes output columns [half * DV / NH, (half + 1) * DV / NH)
+      constexpr int OC = DV / NH;
+      bf16* orow = P.out + flat * DV + half * OC;
+      const uint32_t oaddr = lane_base + LY::TM_O + half * OC;
 #pragma unroll 1
-      for (int c = 0; c < DV / 32; ++c) {
-        uint32_t r[32];
+      for (int c = 0; c < OC / 32; ++c) {
+        uint32_t r[32], r1[32];
         if (have_o) {
           tmem_ld32(oaddr + c * 32, r);
+          if constexpr (NH > 1) tmem_ld32(oaddr + DV + c * 32, r1);
           tmem_ld_wait();
         } else {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) r[k] = 0u;
+          for (int k = 0; k < 32; ++k) r[k] = r1[k] = 0u;
+        }
+        float o[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          o[k] = __uint_as_float(r[k]) * ca;
+          if constexpr (NH > 1) o[k] = fmaf(__uint_as_float(r1[k]), cb, o[k]);
         }
         if (row_ok) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
           for (int k = 0; k < 32; k += 8) {
             uint4 v;
-            v.x = pack_bf16(__uint_as_float(r[k + 0]) * inv, __uint_as_float(r[k + 1]) * inv);
-            v.y = pack_bf16(__uint_as_float(r[k + 2]) * inv, __uint_as_float(r[k + 3]) * inv);
-            v.z = pack_bf16(__uint_as_float(r[k + 4]) * inv, __uint_as_float(r[k + 5]) * inv);
-            v.w = pack_bf16(__uint_as_float(r[k + 6]) * inv, __uint_as_float(r[k + 7]) * inv);
+            v.x = pack_bf16(o[k + 0], o[k + 1]);
+            v.y = pack_bf16(o[k + 2], o[k + 3]);
+            v.z = pack_bf16(o[k + 4], o[k + 5]);
+            v.w = pack_bf16(o[k + 6], o[k + 7]);
             dst[k / 8] = v;
           }
         }
       }
-      if (row_ok && P.row_stat) P.row_stat[flat] = stat;
+      if (row_ok && P.row_stat && half == 0) P.row_stat[flat] = stat;
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, LY::TM_COLS);
+  if (warp == NWN + 1) tmem_dealloc(tmem, LY::TM_COLS);
 }
 
 
