@@ -174,6 +174,22 @@ LAUNCHES = {"softmax": 1, "softmax1": 1, "sparsemax": 3, "entmax15": 3}
 LAUNCHES_DECODE = {"softmax": 2, "softmax1": 2, "sparsemax": 4, "entmax15": 4}
 
 
+def shard_seed(w, rank):
+    """Seed of rank `rank`'s batch: every GPU runs an independent problem of
+    the same shape (weak scaling; the path has no exchange step)."""
+    return w.seed + rank
+
+
+def max_over_ranks(ms, dist, device):
+    """The slowest rank's time: the job finishes when the last rank does."""
+    import torch
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def time_runner(r, steps, warmup, flush):
     """Per-normalizer average kernel time (ms) over `steps` timed steps, each
     preceded by an L2 flush outside the events."""
@@ -298,7 +314,7 @@ def main_native(args):
 
     w = WORKLOADS[args.workload]
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
-    r = Runner(w, dev, seed_offset=rank)
+    r = Runner(w, dev, seed_offset=shard_seed(w, rank) - w.seed)
     for n in w.normalizers:  # warm-up, also the launch configuration checks
         r.call(n)
     torch.cuda.synchronize()
@@ -315,9 +331,7 @@ def main_native(args):
     clocks = sampler.stop()
     ms_step = sum(per.values())
     if world > 1:
-        t = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
+        ms_step = max_over_ranks(ms_step, dist, dev)
         dist.barrier()
 
     units = r.units()
