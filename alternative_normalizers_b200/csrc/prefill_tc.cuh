@@ -50,7 +50,7 @@ constexpr int TC_BM = 128;
 // candidate buffer entries per row in the threshold pass (value + key index)
 template <int D>
 struct TauCap {
-  static constexpr int value = (D >= 256) ? 88 : 112;
+  static constexpr int value = (D >= 256) ? 72 : 96;
 };
 
 struct TcArgs {
@@ -84,7 +84,10 @@ struct TcLayout {
   static constexpr int OFF_BUF = OFF_V + VST * VBYTES;
   static constexpr int CAP = TauCap<D>::value;
   static constexpr int CAP_STRIDE = CAP + 1;  // int2 entries per row
-  static constexpr int BUFBYTES = (MODE == TC_TAU) ? CAP_STRIDE * TC_BM * 8 : 0;
+  // + per-warp staging of one 32-key chunk, [key][lane] floats
+  static constexpr int STAGEBYTES = (MODE == TC_TAU) ? 4 * 32 * 32 * 4 : 0;
+  static constexpr int BUFBYTES = (MODE == TC_TAU) ? CAP_STRIDE * TC_BM * 8 + STAGEBYTES : 0;
+  static constexpr int OFF_STAGE = OFF_BUF + CAP_STRIDE * TC_BM * 8;
   static constexpr int OFF_BAR = OFF_BUF + BUFBYTES;
   static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 2 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -383,6 +386,7 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
     // and exp2(z - m) is one FFMA + EX2 per score
     const bool fast = !(P.softcap > 0.f) && A.zscale > 0.f;
     const float zs = A.zscale;
+    const float izs = 1.f / A.zscale;
 
     float m_run, l_run = 0.f, tau = 0.f;
     // TAU state
@@ -411,21 +415,29 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
         break;
       }
       tc_fence_after();
-      const int j0 = (kb0 + j) * BN + cbase;  // first key of this thread's columns
-      const bool edge = !(rr.lo <= j0 && rr.hi >= j0 + NC - 1);
-      // visible keys of this row inside the block: [kl, kl + span]
-      int kl = rr.lo - j0;
+      const int jb = (kb0 + j) * BN + cbase;  // first key of this thread's columns
+      const bool edge = !(rr.lo <= jb && rr.hi >= jb + NC - 1);
+      // visible keys of this row relative to jb: [klb, klb + span]
+      int klb = rr.lo - jb;
       unsigned span = (unsigned)(rr.hi - rr.lo);
       if (rr.hi < rr.lo) {
-        kl = NC;
+        klb = NC;
         span = 0;
       }
-      const uint32_t saddr = lane_base + (sb ? LY::TM_S1 : LY::TM_S0) + cbase;
+      const uint32_t sbase = lane_base + (sb ? LY::TM_S1 : LY::TM_S0) + cbase;
+      // the online mode needs its whole part of the row at once (maximum
+      // before exponentials); the sparse modes work on 64-key sub-blocks
+      constexpr int LDC = (MODE == TC_ONLINE) ? NC : 64;
+#pragma unroll 1
+      for (int hs = 0; hs < NC / LDC; ++hs) {
+      const uint32_t saddr = sbase + hs * LDC;       // S columns of this sub-block
+      const uint32_t paddr = sbase + hs * (LDC / 2); // packed P columns
+      const int j0 = jb + hs * LDC;
+      const int kl = klb - hs * LDC;
 
-      // this thread's part of the S row, one TMEM round trip
-      uint32_t r[NC];
+      uint32_t r[LDC];
 #pragma unroll
-      for (int c = 0; c < NC / 32; ++c)
+      for (int c = 0; c < LDC / 32; ++c)
         tmem_ld32(saddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
       tmem_ld_wait();
 
@@ -433,18 +445,18 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
       // masked entries become -inf
       if (!fast) {
 #pragma unroll
-        for (int k = 0; k < NC; ++k) r[k] = __float_as_uint(tc_z(__uint_as_float(r[k]), A));
+        for (int k = 0; k < LDC; ++k) r[k] = __float_as_uint(tc_z(__uint_as_float(r[k]), A));
       }
       if (edge) {
 #pragma unroll
-        for (int k = 0; k < NC; ++k)
+        for (int k = 0; k < LDC; ++k)
           if ((unsigned)(k - kl) > span) r[k] = __float_as_uint(-INFINITY);
       }
 
       if constexpr (MODE == TC_ONLINE) {
         float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-        for (int k = 0; k < NC; k += 4) {
+        for (int k = 0; k < LDC; k += 4) {
           mx0 = fmaxf(mx0, __uint_as_float(r[k]));
           mx1 = fmaxf(mx1, __uint_as_float(r[k + 1]));
           mx2 = fmaxf(mx2, __uint_as_float(r[k + 2]));
@@ -460,7 +472,7 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
         const float fa = fast ? zs : 1.f;  // p = exp2(x * fa - msafe)
         float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int c = 0; c < NC / 64; ++c) {  // 64 scores -> 32 packed columns
+        for (int c = 0; c < LDC / 64; ++c) {  // 64 scores -> 32 packed columns
           uint32_t pk[32];
 #pragma unroll
           for (int k = 0; k < 64; k += 2) {
@@ -471,7 +483,7 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
             s1 += p1;
             pk[k >> 1] = pack_bf16(p0, p1);
           }
-          tmem_st32(saddr + c * 32, pk);
+          tmem_st32(paddr + c * 32, pk);
         }
         tmem_st_wait();
         l_run = l_run * alpha + (s0 + s1);
@@ -499,7 +511,7 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
         // p = relu(z - tau) or relu(z/2 - tau)^2 as bf16 P
         const float fa = fast ? zs : 1.f;
 #pragma unroll
-        for (int c = 0; c < NC / 64; ++c) {
+        for (int c = 0; c < LDC / 64; ++c) {
           uint32_t pk[32];
 #pragma unroll
           for (int k = 0; k < 64; k += 2) {
@@ -511,25 +523,39 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
             }
             pk[k >> 1] = pack_bf16(x0, x1);
           }
-          tmem_st32(saddr + c * 32, pk);
+          tmem_st32(paddr + c * 32, pk);
         }
         tmem_st_wait();
       } else {  // TC_TAU
+        // raw scores are compared against the bound mapped back to raw units
+        // (fast path); appending a key a rounding step below the bound is
+        // harmless, the exact solve discards it
+        float* stage = reinterpret_cast<float*>(smem + LY::OFF_STAGE) + quarter * 32 * 32;
 #pragma unroll
-        for (int c = 0; c < NC / 32; ++c) {
-          float cmax = -INFINITY;
+        for (int c = 0; c < LDC / 32; ++c) {
+          float cm0 = -INFINITY, cm1 = -INFINITY;
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            if (fast) r[c * 32 + k] = __float_as_uint(__uint_as_float(r[c * 32 + k]) * zs);
-            cmax = fmaxf(cmax, __uint_as_float(r[c * 32 + k]));
+          for (int k = 0; k < 32; k += 2) {
+            cm0 = fmaxf(cm0, __uint_as_float(r[c * 32 + k]));
+            cm1 = fmaxf(cm1, __uint_as_float(r[c * 32 + k + 1]));
           }
+          const float cmax = fast ? fmaxf(cm0, cm1) * zs : fmaxf(cm0, cm1);
           m_run = fmaxf(m_run, cmax);
           lb = fmaxf(lb, m_run - 1.f);  // tau >= max - 1
           const bool want = cmax > lb && !ovf;
-          // rows whose buffer could overflow on this chunk: raise their
-          // bound to the exact threshold of the keys seen so far (adding keys
-          // only raises tau), then compact; the whole warp works on one row
-          unsigned need = __ballot_sync(0xffffffffu, want && nbuf + 32 > LY::CAP);
+          float thr = fast ? lb * izs : lb;
+          thr = thr - fabsf(thr) * 1e-6f - 1e-30f;  // never above the bound
+          unsigned mask = 0u;
+          if (want) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (__uint_as_float(r[c * 32 + k]) > thr) mask |= 1u << k;
+          }
+          // rows whose buffer could overflow: raise their bound to the exact
+          // threshold of the keys seen so far (adding keys only raises tau),
+          // compact, and re-select this chunk's candidates; one row at a
+          // time with the whole warp
+          unsigned need = __ballot_sync(0xffffffffu, nbuf + __popc(mask) > LY::CAP);
           while (need) {
             const int rr_ = __ffs(need) - 1;
             need &= need - 1;
@@ -541,26 +567,37 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
             const float nlb = warp_row_tau(ent, m_r, entmax, lb_r - m_r);
             const int kept = warp_compact_row(ent, rowp, nlb);
             if (lane == rr_) {
-              lb = nlb;
+              lb = fmaxf(lb, nlb);
               nbuf = kept;
+              float t2 = fast ? lb * izs : lb;
+              t2 = t2 - fabsf(t2) * 1e-6f - 1e-30f;
+              mask = 0u;
+#pragma unroll
+              for (int k = 0; k < 32; ++k)
+                if (__uint_as_float(r[c * 32 + k]) > t2) mask |= 1u << k;
             }
           }
-          if (want && cmax > lb) {
+          if (__any_sync(0xffffffffu, mask != 0u)) {
+            // stage the chunk so the set bits can be visited by index
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              const float u = __uint_as_float(r[c * 32 + k]);
-              if (u > lb) {
-                if (nbuf < LY::CAP) {
-                  mybuf[nbuf] = make_int2(j0 + c * 32 + k, __float_as_int(u));
-                  ++nbuf;
-                } else {
-                  ovf = true;
-                }
+            for (int k = 0; k < 32; ++k) stage[k * 32 + lane] = __uint_as_float(r[c * 32 + k]);
+            __syncwarp();
+            while (mask) {
+              const int k = __ffs(mask) - 1;
+              mask &= mask - 1;
+              const float sv = stage[k * 32 + lane];
+              if (nbuf < LY::CAP) {
+                mybuf[nbuf++] = make_int2(j0 + c * 32 + k, __float_as_int(fast ? sv * zs : sv));
+              } else {
+                ovf = true;
               }
             }
+            __syncwarp();
           }
         }
       }
+      }  // sub-blocks
+      if (!alive) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_pfull(sb));
