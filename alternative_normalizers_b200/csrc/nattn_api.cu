@@ -315,8 +315,11 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
   A.sup_cap = pl.sup_cap;
   if (cudaMemsetAsync(A.ovf_count, 0, sizeof(int), st) != cudaSuccess) return NATTN_ECUDA;
   {
-    using LY = TcLayout<D, D, BN, 2, 1, TC_TAU>;
-    auto k = prefill_tc_kernel<D, D, BN, 2, 1, TC_TAU>;
+    // whole rows per thread: splitting rows halves each buffer, and the
+    // larger buffers measured faster for the wider 1.5-entmax supports
+    constexpr int NHT = 1;
+    using LY = TcLayout<D, D, BN, 2, 1, TC_TAU, NHT>;
+    auto k = prefill_tc_kernel<D, D, BN, 2, 1, TC_TAU, NHT>;
     if (allow_smem(k, LY::ALLOC) != cudaSuccess) return NATTN_ECUDA;
     k<<<grid, LY::THREADS, LY::ALLOC, st>>>(mq, mk, mv, A);
     if (check_launch() != NATTN_OK) return NATTN_ECUDA;

@@ -50,7 +50,7 @@ constexpr int TC_BM = 128;
 // candidate buffer entries per row in the threshold pass (value + key index)
 template <int D>
 struct TauCap {
-  static constexpr int value = (D >= 256) ? 72 : 96;
+  static constexpr int value = (D >= 256) ? 88 : 112;
 };
 
 struct TcArgs {
@@ -72,7 +72,7 @@ struct TcArgs {
 // thread holds half a row in registers.
 template <int D, int DV, int BN, int KST, int VST, int MODE, int NH = 1>
 struct TcLayout {
-  static_assert(NH == 1 || MODE == TC_ONLINE, "row split is for the online mode");
+  static_assert(NH == 1 || MODE != TC_APPLY, "row split is for the online and tau modes");
   static constexpr int NWN = 4 * NH;                 // normalizer warps
   static constexpr int THREADS = (NWN + 2) * 32;     // + TMA warp + MMA warp
   static constexpr int QBYTES = D * TC_BM * 2;
@@ -83,11 +83,9 @@ struct TcLayout {
   static constexpr int OFF_V = OFF_K + KST * KBYTES;
   static constexpr int OFF_BUF = OFF_V + VST * VBYTES;
   static constexpr int CAP = TauCap<D>::value;
-  static constexpr int CAP_STRIDE = CAP + 1;  // int2 entries per row
-  // + per-warp staging of one 32-key chunk, [key][lane] floats
-  static constexpr int STAGEBYTES = (MODE == TC_TAU) ? 4 * 32 * 32 * 4 : 0;
-  static constexpr int BUFBYTES = (MODE == TC_TAU) ? CAP_STRIDE * TC_BM * 8 + STAGEBYTES : 0;
-  static constexpr int OFF_STAGE = OFF_BUF + CAP_STRIDE * TC_BM * 8;
+  static constexpr int CAPR = CAP / NH;         // entries per row half
+  static constexpr int CAP_STRIDE = CAPR + 1;    // int2 entries per row half
+  static constexpr int BUFBYTES = (MODE == TC_TAU) ? CAP_STRIDE * TC_BM * NH * 8 : 0;
   static constexpr int OFF_BAR = OFF_BUF + BUFBYTES;
   static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 2 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -129,8 +127,10 @@ __device__ __forceinline__ float tc_z(float s, const TcArgs& A) {
 // above it, everything else at or below it); for sparsemax this is Michelot's
 // projection algorithm.
 struct RowEntries {
-  int2 e[4];  // (key index, value bits); value -inf marks an empty slot
+  int2 e[4];  // (key index, stored value bits); -inf marks an empty slot
 };
+// Stored values are raw scores on the fast path (threshold units = raw *
+// vscale) and threshold units otherwise (vscale = 1).
 
 __device__ __forceinline__ RowEntries warp_load_row(const int2* row, int n) {
   const int lane = threadIdx.x & 31;
@@ -143,11 +143,11 @@ __device__ __forceinline__ RowEntries warp_load_row(const int2* row, int n) {
   return r;
 }
 
-__device__ __forceinline__ float warp_row_tau(const RowEntries& r, float m, bool entmax,
-                                              float t0) {
+__device__ __forceinline__ float warp_row_tau(const RowEntries& r, float vscale, float m,
+                                              bool entmax, float t0) {
   float w[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) w[i] = __int_as_float(r.e[i].y) - m;
+  for (int i = 0; i < 4; ++i) w[i] = __int_as_float(r.e[i].y) * vscale - m;
   float t = fmaxf(t0, -1.f);
   for (int it = 0; it < 64; ++it) {
     float cnt = 0.f, s1 = 0.f, s2 = 0.f, wmin = INFINITY;
@@ -185,20 +185,28 @@ __device__ __forceinline__ float warp_row_tau(const RowEntries& r, float m, bool
   return t + m;
 }
 
-// Keep the entries above `lb`, compacted to the front of `row`; returns the
-// new count.  Reads happened in warp_load_row, so writing in place is safe.
-__device__ __forceinline__ int warp_compact_row(const RowEntries& r, int2* row, float lb) {
+// Keep the entries above `lb` (threshold units), compacted to the front of
+// `row`; returns the new count and, in *kept_sum, the sum of the kept stored
+// values.  Reads happened in warp_load_row, so writing in place is safe.
+__device__ __forceinline__ int warp_compact_row(const RowEntries& r, int2* row, float vscale,
+                                                float lb, float* kept_sum) {
   const int lane = threadIdx.x & 31;
   const unsigned below = (1u << lane) - 1u;
   int base = 0;
+  float sum = 0.f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const bool keep = __int_as_float(r.e[i].y) > lb;
+    const float v = __int_as_float(r.e[i].y);
+    const bool keep = v * vscale > lb;
     const unsigned bal = __ballot_sync(0xffffffffu, keep);
-    if (keep) row[base + __popc(bal & below)] = r.e[i];
+    if (keep) {
+      row[base + __popc(bal & below)] = r.e[i];
+      sum += v;
+    }
     base += __popc(bal);
   }
   __syncwarp();
+  *kept_sum = warp_sum(sum);
   return base;
 }
 
@@ -390,10 +398,11 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
 
     float m_run, l_run = 0.f, tau = 0.f;
     // TAU state
-    int2* tbuf = reinterpret_cast<int2*>(smem + LY::OFF_BUF) +
-                 (size_t)(quarter * 32) * LY::CAP_STRIDE;  // this warp's 32 rows
+    int2* const bufbase = reinterpret_cast<int2*>(smem + LY::OFF_BUF);
+    int2* tbuf = bufbase + (size_t)(half * TC_BM + quarter * 32) * LY::CAP_STRIDE;  // 32 rows
     int2* mybuf = tbuf + lane * LY::CAP_STRIDE;
     int nbuf = 0;
+    float bsum = 0.f;  // sum of the stored values in the buffer
     bool ovf = false;
     float lb = -INFINITY;  // lower bound of tau (threshold units)
     if constexpr (MODE == TC_ONLINE) {
@@ -527,10 +536,7 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
         }
         tmem_st_wait();
       } else {  // TC_TAU
-        // raw scores are compared against the bound mapped back to raw units
-        // (fast path); appending a key a rounding step below the bound is
-        // harmless, the exact solve discards it
-        float* stage = reinterpret_cast<float*>(smem + LY::OFF_STAGE) + quarter * 32 * 32;
+        const float vs = fast ? zs : 1.f;  // stored value -> threshold units
 #pragma unroll
         for (int c = 0; c < LDC / 32; ++c) {
           float cm0 = -INFINITY, cm1 = -INFINITY;
@@ -539,23 +545,39 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
             cm0 = fmaxf(cm0, __uint_as_float(r[c * 32 + k]));
             cm1 = fmaxf(cm1, __uint_as_float(r[c * 32 + k + 1]));
           }
-          const float cmax = fast ? fmaxf(cm0, cm1) * zs : fmaxf(cm0, cm1);
+          const float cmax = fmaxf(cm0, cm1) * vs;
           m_run = fmaxf(m_run, cmax);
           lb = fmaxf(lb, m_run - 1.f);  // tau >= max - 1
+          // The buffer B holds every stored key that can still be in the
+          // support, so for the threshold of the keys seen so far
+          //   sparsemax: sum_B (u - tau) <= 1          -> tau >= (sum u - 1)/|B|
+          //   entmax15:  sum_B (u - tau) <= sqrt(|B|)  -> tau >= mean u - 1/sqrt|B|
+          // (Cauchy-Schwarz with sum_S (u - tau)^2 = 1); adding keys only
+          // raises tau, so either is a valid running lower bound.
+          if (nbuf > 0) {
+            const float fn = (float)nbuf;
+            const float su = bsum * vs;
+            lb = fmaxf(lb, entmax ? su / fn - rsqrtf(fn) : (su - 1.f) / fn);
+          }
           const bool want = cmax > lb && !ovf;
           float thr = fast ? lb * izs : lb;
           thr = thr - fabsf(thr) * 1e-6f - 1e-30f;  // never above the bound
-          unsigned mask = 0u;
+          int cnt = 0;
           if (want) {
+            int c0 = 0, c1 = 0, c2 = 0, c3 = 0;
 #pragma unroll
-            for (int k = 0; k < 32; ++k)
-              if (__uint_as_float(r[c * 32 + k]) > thr) mask |= 1u << k;
+            for (int k = 0; k < 32; k += 4) {
+              c0 += __uint_as_float(r[c * 32 + k]) > thr;
+              c1 += __uint_as_float(r[c * 32 + k + 1]) > thr;
+              c2 += __uint_as_float(r[c * 32 + k + 2]) > thr;
+              c3 += __uint_as_float(r[c * 32 + k + 3]) > thr;
+            }
+            cnt = c0 + c1 + c2 + c3;
           }
-          // rows whose buffer could overflow: raise their bound to the exact
-          // threshold of the keys seen so far (adding keys only raises tau),
-          // compact, and re-select this chunk's candidates; one row at a
-          // time with the whole warp
-          unsigned need = __ballot_sync(0xffffffffu, nbuf + __popc(mask) > LY::CAP);
+          // rows whose buffer cannot take this chunk's candidates: raise the
+          // bound to the exact threshold of the keys seen so far and compact;
+          // one row at a time with the whole warp
+          unsigned need = __ballot_sync(0xffffffffu, want && nbuf + cnt > LY::CAPR);
           while (need) {
             const int rr_ = __ffs(need) - 1;
             need &= need - 1;
@@ -564,35 +586,39 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
             const float lb_r = __shfl_sync(0xffffffffu, lb, rr_);
             int2* rowp = tbuf + rr_ * LY::CAP_STRIDE;
             const RowEntries ent = warp_load_row(rowp, n_r);
-            const float nlb = warp_row_tau(ent, m_r, entmax, lb_r - m_r);
-            const int kept = warp_compact_row(ent, rowp, nlb);
+            const float nlb = warp_row_tau(ent, vs, m_r, entmax, lb_r - m_r);
+            float ksum;
+            const int kept = warp_compact_row(ent, rowp, vs, nlb, &ksum);
             if (lane == rr_) {
               lb = fmaxf(lb, nlb);
               nbuf = kept;
-              float t2 = fast ? lb * izs : lb;
-              t2 = t2 - fabsf(t2) * 1e-6f - 1e-30f;
-              mask = 0u;
+              bsum = ksum;
+              thr = fast ? lb * izs : lb;
+              thr = thr - fabsf(thr) * 1e-6f - 1e-30f;
+              int c0 = 0;
 #pragma unroll
-              for (int k = 0; k < 32; ++k)
-                if (__uint_as_float(r[c * 32 + k]) > t2) mask |= 1u << k;
+              for (int k = 0; k < 32; ++k) c0 += __uint_as_float(r[c * 32 + k]) > thr;
+              cnt = c0;
             }
           }
-          if (__any_sync(0xffffffffu, mask != 0u)) {
-            // stage the chunk so the set bits can be visited by index
+          if (want && nbuf + cnt > LY::CAPR) ovf = true;  // support too large
+          if (want && !ovf && cnt > 0) {
+            // stored values are compared in stored units; a key a rounding
+            // step below the bound is harmless (the exact solve drops it)
+            int2* ptr = mybuf + nbuf;
+            const int kj = j0 + c * 32;
+            float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-            for (int k = 0; k < 32; ++k) stage[k * 32 + lane] = __uint_as_float(r[c * 32 + k]);
-            __syncwarp();
-            while (mask) {
-              const int k = __ffs(mask) - 1;
-              mask &= mask - 1;
-              const float sv = stage[k * 32 + lane];
-              if (nbuf < LY::CAP) {
-                mybuf[nbuf++] = make_int2(j0 + c * 32 + k, __float_as_int(fast ? sv * zs : sv));
-              } else {
-                ovf = true;
+            for (int k = 0; k < 32; ++k) {
+              const float v = __uint_as_float(r[c * 32 + k]);
+              if (v > thr) {
+                *ptr = make_int2(kj + k, __float_as_int(v));
+                ++ptr;
+                if (k & 1) s1 += v; else s0 += v;
               }
             }
-            __syncwarp();
+            nbuf += cnt;
+            bsum += s0 + s1;
           }
         }
       }
@@ -606,16 +632,39 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
     // ---- epilogue ----------------------------------------------------------
     if constexpr (MODE == TC_TAU) {
       // exact tau and the support list of every row, one row at a time with
-      // the whole warp
-      __syncwarp();
-      for (int rr_ = 0; rr_ < 32; ++rr_) {
-        const int qr = q0 + warp * 32 + rr_;
+      // the whole warp; with split rows the two halves' buffers are merged
+      // (each half's bound is a valid bound of the whole row's threshold)
+      float4* xs = reinterpret_cast<float4*>(smem + LY::OFF_Q);  // Q is no longer read
+      if constexpr (NH > 1) {
+        xs[half * TC_BM + row] = make_float4(m_run, lb, __int_as_float(nbuf), ovf ? 1.f : 0.f);
+        asm volatile("bar.sync 1, %0;" ::"r"(NWN * 32) : "memory");
+      } else {
+        __syncwarp();
+      }
+      constexpr int RPW = 32 / NH;  // rows this warp finishes
+      const float vs = fast ? zs : 1.f;
+      for (int i = 0; i < RPW; ++i) {
+        const int rloc = half * RPW + i;          // row within the quarter
+        const int rq = quarter * 32 + rloc;       // row within the tile
+        const int qr = q0 + rq;
         if (qr >= P.Tq) break;
         const size_t fr = (size_t)bh * P.Tq + qr;
-        const int n_r = __shfl_sync(0xffffffffu, nbuf, rr_);
-        const float m_r = __shfl_sync(0xffffffffu, m_run, rr_);
-        const float lb_r = __shfl_sync(0xffffffffu, lb, rr_);
-        const bool ovf_r = __shfl_sync(0xffffffffu, (int)ovf, rr_) != 0;
+        float m_r, lb_r;
+        int n0, n1 = 0;
+        bool ovf_r;
+        if constexpr (NH > 1) {
+          const float4 a0 = xs[rq], a1 = xs[TC_BM + rq];
+          m_r = fmaxf(a0.x, a1.x);
+          lb_r = fmaxf(a0.y, a1.y);
+          n0 = __float_as_int(a0.z);
+          n1 = __float_as_int(a1.z);
+          ovf_r = a0.w != 0.f || a1.w != 0.f;
+        } else {
+          m_r = __shfl_sync(0xffffffffu, m_run, rloc);
+          lb_r = __shfl_sync(0xffffffffu, lb, rloc);
+          n0 = __shfl_sync(0xffffffffu, nbuf, rloc);
+          ovf_r = __shfl_sync(0xffffffffu, (int)ovf, rloc) != 0;
+        }
         float t = INFINITY;
         int nsup = 0;
         if (ovf_r) {
@@ -624,18 +673,27 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
             A.ovf_rows[slot] = (int)fr;
           }
         } else if (m_r != -INFINITY) {
-          const RowEntries ent = warp_load_row(tbuf + rr_ * LY::CAP_STRIDE, n_r);
-          t = warp_row_tau(ent, m_r, entmax, lb_r - m_r);
+          const int2* b0 = bufbase + (size_t)rq * LY::CAP_STRIDE;
+          const int2* b1 = bufbase + (size_t)(TC_BM + rq) * LY::CAP_STRIDE;
+          RowEntries ent;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int k = lane + 32 * e;
+            ent.e[e] = (k < n0) ? b0[k]
+                       : (k < n0 + n1) ? b1[k - n0]
+                                       : make_int2(0, __float_as_int(-INFINITY));
+          }
+          t = warp_row_tau(ent, vs, m_r, entmax, lb_r - m_r);
           int2* dst = A.sup_list + fr * (size_t)A.sup_cap;
           const unsigned below = (1u << lane) - 1u;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float x = __int_as_float(ent.e[i].y) - t;
+          for (int e = 0; e < 4; ++e) {
+            const float x = __int_as_float(ent.e[e].y) * vs - t;
             const bool in = x > 0.f;
             const unsigned bal = __ballot_sync(0xffffffffu, in);
             if (in)
               dst[nsup + __popc(bal & below)] =
-                  make_int2(ent.e[i].x, __float_as_int(entmax ? x * x : x));
+                  make_int2(ent.e[e].x, __float_as_int(entmax ? x * x : x));
             nsup += __popc(bal);
           }
         }

@@ -21,6 +21,7 @@ workload on the host cores (the reference arm of this benchmark).
 
 import argparse
 import json
+from dataclasses import replace
 import math
 import os
 import statistics
@@ -313,6 +314,8 @@ def main_native(args):
     binding.lib()
 
     w = WORKLOADS[args.workload]
+    if args.normalizer:
+        w = replace(w, normalizers=(args.normalizer,))
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     r = Runner(w, dev, seed_offset=shard_seed(w, rank) - w.seed)
     for n in w.normalizers:  # warm-up, also the launch configuration checks
@@ -386,7 +389,9 @@ def main_native(args):
             (LAUNCHES_DECODE if w.paged else LAUNCHES)[n]
             for n in w.normalizers),
     }
-    if rank == 0:
+    if rank == 0 and args.quick:
+        print(json.dumps(line), flush=True)
+    elif rank == 0:
         e2e_ms, h2d, d2h = e2e_measure(r, max(3, args.steps // 4), dev)
         e2e_val = units * len(w.normalizers) / (e2e_ms * 1e-3) / (
             1e9 if w.paged else 1e12)
@@ -478,6 +483,11 @@ def main():
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--workload", default="qwen3_8b_prefill")
     p.add_argument("--no-detail", dest="detail", action="store_false")
+    p.add_argument("--normalizer", default=None,
+                   help="time only this normalizer of the workload")
+    p.add_argument("--quick", action="store_true",
+                   help="timed steps only (no e2e, CPU baseline or other "
+                        "workloads): the profiling target")
     args = p.parse_args()
     if args.warmup < 3:
         args.warmup = 3
