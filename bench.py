@@ -316,6 +316,8 @@ def main_native(args):
     w = WORKLOADS[args.workload]
     if args.normalizer:
         w = replace(w, normalizers=(args.normalizer,))
+    if args.batch:
+        w = replace(w, B=args.batch)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     r = Runner(w, dev, seed_offset=shard_seed(w, rank) - w.seed)
     for n in w.normalizers:  # warm-up, also the launch configuration checks
@@ -485,6 +487,9 @@ def main():
     p.add_argument("--no-detail", dest="detail", action="store_false")
     p.add_argument("--normalizer", default=None,
                    help="time only this normalizer of the workload")
+    p.add_argument("--batch", type=int, default=0,
+                   help="override the workload's batch (profiling a smaller "
+                        "case of the same kernel)")
     p.add_argument("--quick", action="store_true",
                    help="timed steps only (no e2e, CPU baseline or other "
                         "workloads): the profiling target")
