@@ -14,6 +14,7 @@
 
 #include "common.cuh"
 #include "decode.cuh"
+#include "prefill_pair.cuh"
 #include "prefill_tc.cuh"
 #include "problem.cuh"
 #include "rowwise.cuh"
@@ -296,6 +297,17 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
     A.sup_count = nullptr;
     A.sup_list = nullptr;
     A.sup_cap = 0;
+    // two query heads of one KV group per CTA, each with its own S and O
+    if constexpr (D <= 128) {
+      if ((a->Hq / a->Hkv) % 2 == 0) {
+        using PL = PairLayout<D, KST, VST>;
+        auto kp = prefill_pair_kernel<D, KST, VST>;
+        if (allow_smem(kp, PL::ALLOC) != cudaSuccess) return NATTN_ECUDA;
+        const unsigned pgrid = (unsigned)((long long)a->B * (a->Hq / 2) * ntq);
+        kp<<<pgrid, PAIR_THREADS, PL::ALLOC, st>>>(mq, mk, mv, A);
+        return check_launch();
+      }
+    }
     // split each S row between two warps where TMEM holds two O halves
     constexpr int NH = (2 * BN + 2 * D <= 512) ? 2 : 1;
     using LY = TcLayout<D, D, BN, KST, VST, TC_ONLINE, NH>;

@@ -1,0 +1,392 @@
+// Online softmax / softmax1 prefill with two query tiles per CTA.
+//
+// The CTA takes the same 128 query rows of two query heads that read the same
+// key/value head (grouped-query attention with an even group), so both tiles
+// walk the same visible key blocks and every K/V block brought in by TMA
+// feeds two products.  Each tile owns one S buffer and one O accumulator in
+// TMEM (2 x (128 + 128) = 512 columns) and one normalizer warpgroup.  The
+// single MMA thread interleaves the tiles:
+//
+//     ... PV_A(j)  QK_A(j+1)  PV_B(j)  QK_B(j+1)  PV_A(j+1) ...
+//
+// so while warpgroup A turns S_A(j+1) into P it is the other tile's products
+// that keep the tensor pipe busy, and the hand-off latencies of one tile
+// (S ready -> normalizer, P ready -> PV issue) are covered by the other
+// tile's work.  P is written back over its own S columns; the QK that next
+// overwrites them is issued after the PV that reads them, and tcgen05.mma
+// operations from one thread execute in issue order.
+//
+// softmax1 starts each row from the virtual logit-0 / value-0 sink ("HF
+// Attention Normalizers", section "Important Limitations"): m0 = 0, l0 = 1.
+#pragma once
+
+#include "common.cuh"
+#include "prefill_tc.cuh"
+#include "problem.cuh"
+
+namespace nattn {
+
+constexpr int PAIR_THREADS = 320;  // 8 normalizer warps + TMA warp + MMA warp
+
+template <int D, int KST, int VST>
+struct PairLayout {
+  static constexpr int BN = 128;
+  static constexpr int QBYTES = D * TC_BM * 2;  // one tile
+  static constexpr int KBYTES = D * BN * 2;
+  static constexpr int VBYTES = D * BN * 2;
+  static constexpr int OFF_Q = 0;               // tile 0, then tile 1
+  static constexpr int OFF_K = 2 * QBYTES;
+  static constexpr int OFF_V = OFF_K + KST * KBYTES;
+  static constexpr int OFF_BAR = OFF_V + VST * VBYTES;
+  // q, kfull/kempty, vfull/vempty, sfull[2], pfull[2], pvdone[2]
+  static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 6;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;
+  static constexpr int TM_S = 0;                // tile t: TM_S + t * BN
+  static constexpr int TM_O = 2 * BN;           // tile t: TM_O + t * D
+  static constexpr int TM_COLS = (2 * BN + 2 * D <= 256) ? 256 : 512;
+  static_assert(2 * BN + 2 * D <= 512, "TMEM budget");
+  static_assert(ALLOC <= 227 * 1024, "shared memory budget");
+};
+
+// One normalizer warp of tile t = warp / 4: thread = query row = TMEM lane of
+// its lane quarter.  The S row is read in two 64-column halves twice (maximum,
+// then exponentials), which keeps the register count within the 320-thread
+// budget; TMEM reads are cheap next to the exponentials.
+template <int D, int KST, int VST>
+__device__ __forceinline__ void prefill_pair_normalizer(
+    const TcArgs& A, uint8_t* smem, uint32_t tmem, int warp, int lane, int q0, int bh0,
+    int kb0, int nblk, uint32_t bar_sf, uint32_t bar_pf, uint32_t bar_pvt,
+    volatile int* abort_flag) {
+  using LY = PairLayout<D, KST, VST>;
+  constexpr int BN = LY::BN;
+  const Problem& P = A.P;
+  const int t = warp >> 2, quarter = warp & 3;
+  const int row = quarter * 32 + lane;
+  const int qi = q0 + row;
+  const bool row_ok = qi < P.Tq;
+  RowRange rr = row_range(P, qi, P.Tk);
+  if (!row_ok) rr = RowRange{1, 0};
+  if (rr.hi > P.Tk - 1) rr.hi = P.Tk - 1;
+  const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+  const uint32_t sbase = lane_base + LY::TM_S + t * BN;
+  const uint32_t obase = lane_base + LY::TM_O + t * D;
+  const size_t flat = (size_t)(bh0 + t) * P.Tq + qi;
+  const bool fast = !(P.softcap > 0.f) && A.zscale > 0.f;
+  const float fa = fast ? A.zscale : 1.f;  // p = exp2(x * fa - m)
+  const bool sm1 = P.norm == NATTN_SOFTMAX1;
+  float m_run = sm1 ? 0.f : -INFINITY;
+  float l_run = sm1 ? 1.f : 0.f;
+  bool alive = true;
+
+  for (int j = 0; j < nblk; ++j) {
+    if (!__all_sync(0xffffffffu, mbar_wait_spin(bar_sf, j & 1, abort_flag))) {
+      alive = false;
+      break;
+    }
+    tc_fence_after();
+    const int jb = (kb0 + j) * BN;
+    const bool edge = !(rr.lo <= jb && rr.hi >= jb + BN - 1);
+    int kl = rr.lo - jb;
+    unsigned span = (unsigned)(rr.hi - rr.lo);
+    if (rr.hi < rr.lo) {
+      kl = BN;
+      span = 0;
+    }
+    // scores of one 64-column half -> x (raw on the fast path, else z in
+    // log2 units), masked entries -inf
+    auto load_half = [&](int hh, uint32_t (&r)[64]) {
+      tmem_ld32(sbase + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+      tmem_ld32(sbase + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+      tmem_ld_wait();
+      if (!fast) {
+#pragma unroll
+        for (int k = 0; k < 64; ++k) r[k] = __float_as_uint(tc_z(__uint_as_float(r[k]), A));
+      }
+      if (edge) {
+#pragma unroll
+        for (int k = 0; k < 64; ++k)
+          if ((unsigned)(hh * 64 + k - kl) > span) r[k] = __float_as_uint(-INFINITY);
+      }
+    };
+    float mx = -INFINITY;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      uint32_t r[64];
+      load_half(hh, r);
+      float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < 64; k += 4) {
+        a0 = fmaxf(a0, __uint_as_float(r[k]));
+        a1 = fmaxf(a1, __uint_as_float(r[k + 1]));
+        a2 = fmaxf(a2, __uint_as_float(r[k + 2]));
+        a3 = fmaxf(a3, __uint_as_float(r[k + 3]));
+      }
+      mx = fmaxf(mx, fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)));
+    }
+    mx *= fa;
+    const float mnew = fmaxf(m_run, mx);
+    const bool resc = mnew > m_run + 8.f;  // move the maximum only when it grows by 2^8
+    const float m_use = resc ? mnew : m_run;
+    const float alpha = resc ? fast_exp2(m_run - mnew) : 1.f;
+    const float msafe = (m_use == -INFINITY) ? 0.f : m_use;
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      uint32_t r[64];
+      load_half(hh, r);
+      uint32_t pk[32];
+#pragma unroll
+      for (int k = 0; k < 64; k += 2) {
+        const float p0 = fast_exp2(fmaf(__uint_as_float(r[k]), fa, -msafe));
+        const float p1 = fast_exp2(fmaf(__uint_as_float(r[k + 1]), fa, -msafe));
+        s0 += p0;
+        s1 += p1;
+        pk[k >> 1] = pack_bf16(p0, p1);
+      }
+      // packed P of keys [64 hh, 64 hh + 64) over S columns already read
+      tmem_st32(sbase + hh * 32, pk);
+    }
+    tmem_st_wait();
+    l_run = l_run * alpha + (s0 + s1);
+    if (__any_sync(0xffffffffu, resc) && j > 0) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_pvt, (j - 1) & 1, abort_flag))) {
+        alive = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(obase + c * 32, o);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+        tmem_st32(obase + c * 32, o);
+      }
+      tmem_st_wait();
+    }
+    m_run = m_use;
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_pf);
+  }
+
+  // ---- epilogue -------------------------------------------------------------
+  const bool have_o = __all_sync(
+      0xffffffffu, alive && nblk > 0 && mbar_wait(bar_pvt, (nblk - 1) & 1, abort_flag));
+  tc_fence_after();
+  const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+  const float msafe = (m_run == -INFINITY) ? 0.f : m_run;
+  const float stat = (l_run > 0.f) ? (msafe + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+  bf16* orow = P.out + flat * D;
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t r[32];
+    if (have_o) {
+      tmem_ld32(obase + c * 32, r);
+      tmem_ld_wait();
+    } else {
+#pragma unroll
+      for (int k = 0; k < 32; ++k) r[k] = 0u;
+    }
+    if (row_ok) {
+      uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+      for (int k = 0; k < 32; k += 8) {
+        uint4 v;
+        v.x = pack_bf16(__uint_as_float(r[k + 0]) * inv, __uint_as_float(r[k + 1]) * inv);
+        v.y = pack_bf16(__uint_as_float(r[k + 2]) * inv, __uint_as_float(r[k + 3]) * inv);
+        v.z = pack_bf16(__uint_as_float(r[k + 4]) * inv, __uint_as_float(r[k + 5]) * inv);
+        v.w = pack_bf16(__uint_as_float(r[k + 6]) * inv, __uint_as_float(r[k + 7]) * inv);
+        dst[k / 8] = v;
+      }
+    }
+  }
+  if (row_ok && P.row_stat) P.row_stat[flat] = stat;
+}
+
+template <int D, int KST, int VST>
+__global__ void __launch_bounds__(PAIR_THREADS, 1)
+    prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq,
+                        const __grid_constant__ CUtensorMap tmk,
+                        const __grid_constant__ CUtensorMap tmv, TcArgs A) {
+  using LY = PairLayout<D, KST, VST>;
+  constexpr int BN = LY::BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const Problem& P = A.P;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ---- tile selection: (query tile, batch, pair of heads of one group) ---
+  const int ntq = (P.Tq + TC_BM - 1) / TC_BM;
+  const int HP = P.Hq / 2;                 // head pairs per batch
+  const int BP = P.B * HP;
+  const int rank = blockIdx.x;
+  const int qt = P.causal ? (ntq - 1 - rank / BP) : (rank / BP);
+  const int bp = rank % BP;
+  const int b = bp / HP;
+  const int h0 = 2 * (bp % HP);
+  const int g = h0 / (P.Hq / P.Hkv);
+  const int bh0 = b * P.Hq + h0;           // tile t reads query head h0 + t
+  const int q0 = qt * TC_BM;
+  const int qlast = min(q0 + TC_BM - 1, P.Tq - 1);
+  const RowRange r_first = row_range(P, q0, P.Tk);
+  const RowRange r_last = row_range(P, qlast, P.Tk);
+  const int klo = max(0, r_first.lo);
+  const int khi = min(P.Tk - 1, r_last.hi);
+  const int kb0 = klo / BN;
+  const int nblk = (khi >= klo) ? (khi / BN - kb0 + 1) : 0;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + LY::OFF_BAR);
+  const uint32_t bar_q = smem_addr(&bars[0]);
+  auto bar_kfull = [&](int s) { return smem_addr(&bars[1 + s]); };
+  auto bar_kempty = [&](int s) { return smem_addr(&bars[1 + KST + s]); };
+  auto bar_vfull = [&](int s) { return smem_addr(&bars[1 + 2 * KST + s]); };
+  auto bar_vempty = [&](int s) { return smem_addr(&bars[1 + 2 * KST + VST + s]); };
+  auto bar_sfull = [&](int t) { return smem_addr(&bars[1 + 2 * KST + 2 * VST + t]); };
+  auto bar_pfull = [&](int t) { return smem_addr(&bars[1 + 2 * KST + 2 * VST + 2 + t]); };
+  auto bar_pv = [&](int t) { return smem_addr(&bars[1 + 2 * KST + 2 * VST + 4 + t]); };
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + LY::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
+
+  if (tid == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < KST; ++s) {
+      mbar_init(bar_kfull(s), 1);
+      mbar_init(bar_kempty(s), 1);
+    }
+    for (int s = 0; s < VST; ++s) {
+      mbar_init(bar_vfull(s), 1);
+      mbar_init(bar_vempty(s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar_sfull(t), 1);
+      mbar_init(bar_pfull(t), 4);
+      mbar_init(bar_pv(t), 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_addr(&misc[0]), LY::TM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  if (warp == 8) {
+    // ======================= TMA producer ===================================
+    if (lane == 0 && nblk > 0) {
+      tma_prefetch_desc(&tmq);
+      tma_prefetch_desc(&tmk);
+      tma_prefetch_desc(&tmv);
+      mbar_expect_tx(bar_q, 2 * LY::QBYTES);
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int x = 0; x < D / 64; ++x)
+          tma_load_3d(smem_addr(smem + LY::OFF_Q + t * LY::QBYTES + x * TC_BM * 128), &tmq,
+                      bar_q, x * 64, q0, bh0 + t);
+      for (int j = 0; j < nblk; ++j) {
+        const int kb = kb0 + j;
+        const int ks = j % KST;
+        if (j >= KST && !mbar_wait(bar_kempty(ks), ((j / KST) + 1) & 1, abort_flag)) break;
+        mbar_expect_tx(bar_kfull(ks), LY::KBYTES);
+        uint8_t* kdst = smem + LY::OFF_K + ks * LY::KBYTES;
+#pragma unroll
+        for (int x = 0; x < D / 64; ++x)
+          tma_load_3d(smem_addr(kdst + x * BN * 128), &tmk, bar_kfull(ks), x * 64, kb * BN,
+                      b * P.Hkv + g);
+        const int vs = j % VST;
+        if (j >= VST && !mbar_wait(bar_vempty(vs), ((j / VST) + 1) & 1, abort_flag)) break;
+        mbar_expect_tx(bar_vfull(vs), LY::VBYTES);
+        uint8_t* vdst = smem + LY::OFF_V + vs * LY::VBYTES;
+#pragma unroll
+        for (int x = 0; x < D / 64; ++x)
+          tma_load_3d(smem_addr(vdst + x * BN * 128), &tmv, bar_vfull(vs), x * 64, kb * BN,
+                      b * P.Hkv + g);
+      }
+    }
+  } else if (warp == 9) {
+    // ======================= MMA issuer =====================================
+    if (lane == 0 && nblk > 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16(TC_BM, BN, 0, 0);
+      constexpr uint32_t IDESC_O = idesc_bf16(TC_BM, D, 0, 1);
+      bool ok = mbar_wait_spin(bar_q, 0, abort_flag);
+      tc_fence_after();
+      auto issue_qk = [&](int t, int j) {
+        const uint32_t qbase = smem_addr(smem + LY::OFF_Q + t * LY::QBYTES);
+        const uint32_t kbase = smem_addr(smem + LY::OFF_K + (j % KST) * LY::KBYTES);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad =
+              sdesc_sw128(qbase + (kk >> 2) * TC_BM * 128 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(kbase + (kk >> 2) * BN * 128 + (kk & 3) * 32, 16, 1024);
+          umma_ss(tmem + LY::TM_S + t * BN, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar_sfull(t));
+      };
+      // prologue: both tiles' scores of the first block
+      if (ok && mbar_wait_spin(bar_kfull(0), 0, abort_flag)) {
+        tc_fence_after();
+        issue_qk(0, 0);
+        issue_qk(1, 0);
+        umma_commit(bar_kempty(0));
+      } else {
+        ok = false;
+      }
+      for (int j = 0; ok && j < nblk; ++j) {
+        const int vs = j % VST;
+        if (!mbar_wait_spin(bar_vfull(vs), (j / VST) & 1, abort_flag)) break;
+        bool k_next = false;
+        for (int t = 0; t < 2; ++t) {
+          if (!mbar_wait_spin(bar_pfull(t), j & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t vbase = smem_addr(smem + LY::OFF_V + vs * LY::VBYTES);
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            // V block [BN keys][D] in 64-column boxes: MN-major B operand
+            const uint64_t bd = sdesc_sw128(vbase + kk * 16 * 128, BN * 128, 1024);
+            umma_ts(tmem + LY::TM_O + t * D, tmem + LY::TM_S + t * BN + kk * 8, bd, IDESC_O,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(bar_pv(t));
+          if (t == 1) umma_commit(bar_vempty(vs));
+          if (j + 1 < nblk) {
+            // this tile's next scores go in behind its PV (issue order)
+            if (t == 0) {
+              if (!mbar_wait_spin(bar_kfull((j + 1) % KST), ((j + 1) / KST) & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              k_next = true;
+            }
+            issue_qk(t, j + 1);
+            if (t == 1 && k_next) umma_commit(bar_kempty((j + 1) % KST));
+          }
+        }
+      }
+    }
+  } else {
+    // normalizer warpgroups: see prefill_pair_normalizer below
+    prefill_pair_normalizer<D, KST, VST>(A, smem, tmem, warp, lane, q0, bh0, kb0, nblk,
+                                         bar_sfull(warp >> 2), bar_pfull(warp >> 2),
+                                         bar_pv(warp >> 2), abort_flag);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9) tmem_dealloc(tmem, LY::TM_COLS);
+}
+
+}  // namespace nattn
