@@ -412,12 +412,98 @@ def main_native(args):
                        "ms_per_step": round(e2e_ms, 3)}
         if world == 1 and not w.paged:
             line["cpu_baseline"] = cpu_baseline_prefill(w, r.host)
-        if args.detail:
+        if args.detail and world == 1:
             line["other_workloads"] = detail(args, dev, flush)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def sparse_prefill_stats(r, n):
+    """Support statistics of one sparse normalizer on a dense workload: the
+    rows' thresholds come from the kernel (row_stat), the scores are
+    recomputed in float32 with torch (measurement only).  Returns the mean
+    threshold, the support size (mean / p99 / max) and the fraction of
+    visible weights that are exactly zero."""
+    import torch
+    w = r.w
+    r.call(n)
+    if r.stat.is_cuda:
+        torch.cuda.synchronize()
+    tau = r.stat.float()
+    half = 0.5 if n == "entmax15" else 1.0
+    sup_all, vis_all = [], 0
+    ii = torch.arange(w.Tq, device=tau.device)[:, None]
+    jj = torch.arange(w.Tk, device=tau.device)[None, :]
+    off = w.Tk - w.Tq
+    allowed = torch.ones(w.Tq, w.Tk, dtype=torch.bool, device=tau.device)
+    if w.causal:
+        allowed &= jj <= ii + off
+    if w.window > 0:
+        allowed &= jj > ii + off - w.window
+    vis_all = int(allowed.sum()) * w.B * w.Hq
+    grp = w.Hq // w.Hkv
+    for b in range(w.B):
+        for h in range(w.Hq):
+            q = r.x["q"][b, h].float()
+            k = r.x["k"][b, h // grp].float()
+            z = (q @ k.T) * w.scale
+            if w.softcap > 0:
+                z = w.softcap * torch.tanh(z / w.softcap)
+            u = z * half
+            u = u.masked_fill(~allowed, float("-inf"))
+            sup_all.append((u > tau[b, h][:, None]).sum(dim=1))
+    sup = torch.cat(sup_all).float()
+    return {"tau_mean": round(float(tau[torch.isfinite(tau)].mean()), 4),
+            "support_mean": round(float(sup.mean()), 2),
+            "support_p99": float(torch.quantile(sup[:1 << 20], 0.99)),
+            "support_max": int(sup.max()),
+            "exact_zero_fraction": round(1.0 - float(sup.sum()) / vis_all, 6)}
+
+
+def sparse_decode_bytes(r, n):
+    """Bytes a sparse decode step actually moves, next to the dense-equivalent
+    K/V count: every K page (the score pass), the fp32 scores written once
+    and read twice (threshold, then apply), the V pages that carry a nonzero
+    weight for some query head of their group, and Q/O.  Which V pages are
+    loaded is recomputed here from the kernel's thresholds and float32
+    scores (measurement only); split partials (under 1 % here) are left
+    out."""
+    import torch
+    w = r.w
+    r.call(n)
+    if r.stat.is_cuda:
+        torch.cuda.synchronize()
+    tau = r.stat.float()
+    half = 0.5 if n == "entmax15" else 1.0
+    grp = w.Hq // w.Hkv
+    ps = w.page_size
+    kb = vb = sb = 0
+    vpages = 0
+    for b in range(w.B):
+        L = int(r.host["seqlens"][b])
+        npg = (L + ps - 1) // ps
+        pages = r.x["block_table"][b, :npg].long()
+        kseq = r.x["k_pool"][pages]                      # [npg, Hkv, ps, d]
+        kseq = kseq.permute(1, 0, 2, 3).reshape(w.Hkv, npg * ps, w.d)[:, :L]
+        q = r.x["q"][b, :, 0].float()                    # [Hq, d]
+        z = torch.einsum("hgd,htd->hgt", q.view(w.Hkv, grp, w.d),
+                         kseq.float()) * w.scale         # [Hkv, grp, L]
+        if w.softcap > 0:
+            z = w.softcap * torch.tanh(z / w.softcap)
+        t = tau[b, :, 0].view(w.Hkv, grp, 1)
+        hit = (z * half > t).any(dim=1)                  # [Hkv, L]
+        pad = npg * ps - L
+        if pad:
+            hit = torch.nn.functional.pad(hit, (0, pad))
+        vpages += int(hit.view(w.Hkv, npg, ps).any(dim=2).sum())
+        kb += npg * ps * w.Hkv * w.d * 2
+        sb += 3 * w.Hq * L * 4
+    vb = vpages * ps * w.dv * 2
+    qo = w.B * w.Hq * (w.d + w.dv) * 2
+    return {"k_bytes": kb, "v_bytes": vb, "score_bytes": sb, "qo_bytes": qo,
+            "total": kb + vb + sb + qo, "v_pages": vpages}
 
 
 def detail(args, dev, flush):
@@ -441,6 +527,19 @@ def detail(args, dev, flush):
                 unit = "useful TFLOP/s"
             res[name] = {"unit": unit, "value": vals,
                          "ms": {n: round(t, 4) for n, t in per.items()}}
+            sparse = [n for n in per if n in ("sparsemax", "entmax15")]
+            if w.paged and sparse:
+                peak = load_peaks()[0]["hbm_gbs"]
+                act = {}
+                for n in sparse:
+                    by = sparse_decode_bytes(r, n)
+                    gbs = by["total"] / (per[n] * 1e-3) / 1e9
+                    act[n] = {"GB/s": round(gbs, 1), "bytes": by,
+                              "frac_of_hbm": round(gbs / peak, 4)}
+                res[name]["actual_bytes"] = act
+            elif sparse:
+                res[name]["support"] = {n: sparse_prefill_stats(r, n)
+                                        for n in sparse}
             del r
             torch.cuda.empty_cache()
         except Exception as exc:  # report, keep the headline line
