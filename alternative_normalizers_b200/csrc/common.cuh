@@ -62,6 +62,24 @@ __device__ __forceinline__ float fast_tanh(float x) {
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// Three-input maximum (sm_100 `max.f32` with three sources).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float y;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+  return y;
+}
+// Maximum of 32 consecutive values held as raw bits (two three-input chains
+// and a final merge: 16 instructions instead of 31 two-input ones).
+__device__ __forceinline__ float max32_bits(const uint32_t* v) {
+  float a = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
+  float b = fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5]));
+#pragma unroll
+  for (int k = 6; k < 30; k += 4) {
+    a = fmax3(a, __uint_as_float(v[k]), __uint_as_float(v[k + 1]));
+    b = fmax3(b, __uint_as_float(v[k + 2]), __uint_as_float(v[k + 3]));
+  }
+  return fmax3(a, b, fmaxf(__uint_as_float(v[30]), __uint_as_float(v[31])));
+}
 
 // ---------------------------------------------------------------------------
 // Shared memory addresses and mbarriers

@@ -72,7 +72,7 @@ struct TcArgs {
 // thread holds half a row in registers.
 template <int D, int DV, int BN, int KST, int VST, int MODE, int NH = 1>
 struct TcLayout {
-  static_assert(NH == 1 || MODE != TC_APPLY, "row split is for the online and tau modes");
+  static_assert(NH == 1 || MODE == TC_ONLINE, "row split is for the online mode");
   static constexpr int NWN = 4 * NH;                 // normalizer warps
   static constexpr int THREADS = (NWN + 2) * 32;     // + TMA warp + MMA warp
   static constexpr int QBYTES = D * TC_BM * 2;
@@ -114,10 +114,11 @@ __device__ __forceinline__ float tc_z(float s, const TcArgs& A) {
   return s * A.zscale;
 }
 
-// Exact threshold of one row's candidate buffer, computed by the whole warp
-// (every lane holds up to four entries of that row in registers).  Values are
-// in threshold units u; `m` is the row maximum, `t0` a lower bound of tau in
-// shifted units (u - m).
+// Exact threshold of one row's candidate buffer, computed by the thread that
+// owns the row (the 32 rows of a warp are solved side by side).  Stored
+// values are raw scores on the fast path (threshold units = raw * vscale) and
+// threshold units otherwise (vscale = 1); `m` is the row maximum and `t0` a
+// lower bound of tau in shifted units (u - m).
 //
 // Newton's method from the left on g(t) = sum relu(u - t)^k - 1 (k = 1 for
 // sparsemax, 2 for 1.5-entmax), which is convex and decreasing, so every
@@ -126,44 +127,21 @@ __device__ __forceinline__ float tc_z(float s, const TcArgs& A) {
 // first and accepted once it satisfies the optimality conditions (all members
 // above it, everything else at or below it); for sparsemax this is Michelot's
 // projection algorithm.
-struct RowEntries {
-  int2 e[4];  // (key index, stored value bits); -inf marks an empty slot
-};
-// Stored values are raw scores on the fast path (threshold units = raw *
-// vscale) and threshold units otherwise (vscale = 1).
-
-__device__ __forceinline__ RowEntries warp_load_row(const int2* row, int n) {
-  const int lane = threadIdx.x & 31;
-  RowEntries r;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int k = lane + 32 * i;
-    r.e[i] = (k < n) ? row[k] : make_int2(0, __float_as_int(-INFINITY));
-  }
-  return r;
-}
-
-__device__ __forceinline__ float warp_row_tau(const RowEntries& r, float vscale, float m,
-                                              bool entmax, float t0) {
-  float w[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) w[i] = __int_as_float(r.e[i].y) * vscale - m;
+__device__ __forceinline__ float thread_row_tau(const int2* row, int n, float vscale, float m,
+                                                bool entmax, float t0) {
   float t = fmaxf(t0, -1.f);
   for (int it = 0; it < 64; ++it) {
     float cnt = 0.f, s1 = 0.f, s2 = 0.f, wmin = INFINITY;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (w[i] > t) {
+#pragma unroll 4
+    for (int i = 0; i < n; ++i) {
+      const float w = __int_as_float(row[i].y) * vscale - m;
+      if (w > t) {
         cnt += 1.f;
-        s1 += w[i];
-        s2 += w[i] * w[i];
-        wmin = fminf(wmin, w[i]);
+        s1 += w;
+        s2 = fmaf(w, w, s2);
+        wmin = fminf(wmin, w);
       }
     }
-    cnt = warp_sum(cnt);
-    s1 = warp_sum(s1);
-    s2 = warp_sum(s2);
-    wmin = warp_min(wmin);
     float ts, tn;
     bool valid = true;
     if (!entmax) {
@@ -185,29 +163,23 @@ __device__ __forceinline__ float warp_row_tau(const RowEntries& r, float vscale,
   return t + m;
 }
 
-// Keep the entries above `lb` (threshold units), compacted to the front of
-// `row`; returns the new count and, in *kept_sum, the sum of the kept stored
-// values.  Reads happened in warp_load_row, so writing in place is safe.
-__device__ __forceinline__ int warp_compact_row(const RowEntries& r, int2* row, float vscale,
-                                                float lb, float* kept_sum) {
-  const int lane = threadIdx.x & 31;
-  const unsigned below = (1u << lane) - 1u;
-  int base = 0;
+// Keep the entries above `lb` (threshold units), compacted in place to the
+// front of the row; returns the new count and, in *kept_sum, the sum of the
+// kept stored values.
+__device__ __forceinline__ int thread_compact_row(int2* row, int n, float vscale, float lb,
+                                                  float* kept_sum) {
+  int j = 0;
   float sum = 0.f;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float v = __int_as_float(r.e[i].y);
-    const bool keep = v * vscale > lb;
-    const unsigned bal = __ballot_sync(0xffffffffu, keep);
-    if (keep) {
-      row[base + __popc(bal & below)] = r.e[i];
+  for (int i = 0; i < n; ++i) {
+    const int2 e = row[i];
+    const float v = __int_as_float(e.y);
+    if (v * vscale > lb) {
+      row[j++] = e;
       sum += v;
     }
-    base += __popc(bal);
   }
-  __syncwarp();
-  *kept_sum = warp_sum(sum);
-  return base;
+  *kept_sum = sum;
+  return j;
 }
 
 template <int D, int DV, int BN, int KST, int VST, int MODE, int NH = 1>
@@ -539,13 +511,8 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
         const float vs = fast ? zs : 1.f;  // stored value -> threshold units
 #pragma unroll
         for (int c = 0; c < LDC / 32; ++c) {
-          float cm0 = -INFINITY, cm1 = -INFINITY;
-#pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            cm0 = fmaxf(cm0, __uint_as_float(r[c * 32 + k]));
-            cm1 = fmaxf(cm1, __uint_as_float(r[c * 32 + k + 1]));
-          }
-          const float cmax = fmaxf(cm0, cm1) * vs;
+          const uint32_t* rc = &r[c * 32];
+          const float cmax = max32_bits(rc) * vs;
           m_run = fmaxf(m_run, cmax);
           lb = fmaxf(lb, m_run - 1.f);  // tau >= max - 1
           // The buffer B holds every stored key that can still be in the
@@ -557,68 +524,65 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
           if (nbuf > 0) {
             const float fn = (float)nbuf;
             const float su = bsum * vs;
-            lb = fmaxf(lb, entmax ? su / fn - rsqrtf(fn) : (su - 1.f) / fn);
+            lb = fmaxf(lb, entmax ? __fdividef(su, fn) - rsqrtf(fn) : __fdividef(su - 1.f, fn));
           }
           const bool want = cmax > lb && !ovf;
-          float thr = fast ? lb * izs : lb;
-          thr = thr - fabsf(thr) * 1e-6f - 1e-30f;  // never above the bound
-          int cnt = 0;
-          if (want) {
-            int c0 = 0, c1 = 0, c2 = 0, c3 = 0;
+          if (!__any_sync(0xffffffffu, want)) continue;
+          // candidates are tested in stored units against the bound less a
+          // margin far above the rounding of the bound's arithmetic
+          auto to_thr = [&](float b) {
+            const float bm = b - (fabsf(b) + 1.f) * 4e-6f;
+            return fast ? bm * izs : bm;
+          };
+          float thr = to_thr(lb);
+          // candidate mask: bit k set when value k is above thr, taken from
+          // the sign of thr - v (-inf values give +inf: never candidates)
+          auto cand_mask = [&](float t) {
+            unsigned mk = 0;
 #pragma unroll
-            for (int k = 0; k < 32; k += 4) {
-              c0 += __uint_as_float(r[c * 32 + k]) > thr;
-              c1 += __uint_as_float(r[c * 32 + k + 1]) > thr;
-              c2 += __uint_as_float(r[c * 32 + k + 2]) > thr;
-              c3 += __uint_as_float(r[c * 32 + k + 3]) > thr;
-            }
-            cnt = c0 + c1 + c2 + c3;
-          }
-          // rows whose buffer cannot take this chunk's candidates: raise the
-          // bound to the exact threshold of the keys seen so far and compact;
-          // one row at a time with the whole warp
-          unsigned need = __ballot_sync(0xffffffffu, want && nbuf + cnt > LY::CAPR);
-          while (need) {
-            const int rr_ = __ffs(need) - 1;
-            need &= need - 1;
-            const int n_r = __shfl_sync(0xffffffffu, nbuf, rr_);
-            const float m_r = __shfl_sync(0xffffffffu, m_run, rr_);
-            const float lb_r = __shfl_sync(0xffffffffu, lb, rr_);
-            int2* rowp = tbuf + rr_ * LY::CAP_STRIDE;
-            const RowEntries ent = warp_load_row(rowp, n_r);
-            const float nlb = warp_row_tau(ent, vs, m_r, entmax, lb_r - m_r);
-            float ksum;
-            const int kept = warp_compact_row(ent, rowp, vs, nlb, &ksum);
-            if (lane == rr_) {
-              lb = fmaxf(lb, nlb);
-              nbuf = kept;
-              bsum = ksum;
-              thr = fast ? lb * izs : lb;
-              thr = thr - fabsf(thr) * 1e-6f - 1e-30f;
-              int c0 = 0;
-#pragma unroll
-              for (int k = 0; k < 32; ++k) c0 += __uint_as_float(r[c * 32 + k]) > thr;
-              cnt = c0;
+            for (int k = 31; k >= 0; --k)
+              mk = __funnelshift_l(__float_as_uint(t - __uint_as_float(rc[k])), mk, 1);
+            return mk;
+          };
+          unsigned msk = want ? cand_mask(thr) : 0u;
+          int cnt = __popc(msk);
+          // when a row's buffer cannot take this chunk's candidates, every row
+          // of the warp raises its bound to the exact threshold of the keys
+          // it has seen and compacts (each thread its own row, side by side:
+          // the rows of a tile fill their buffers at similar rates, so one
+          // batch stands in for many single-row solves)
+          if (__any_sync(0xffffffffu, nbuf + cnt > LY::CAPR)) {
+            lb = fmaxf(lb, thread_row_tau(mybuf, nbuf, vs, m_run, entmax, lb - m_run));
+            nbuf = thread_compact_row(mybuf, nbuf, vs, lb, &bsum);
+            thr = to_thr(lb);
+            msk = want ? cand_mask(thr) : 0u;
+            cnt = __popc(msk);
+            if (nbuf + cnt > LY::CAPR) {  // support too large for the buffer
+              ovf = true;
+              msk = 0;
+              cnt = 0;
             }
           }
-          if (want && nbuf + cnt > LY::CAPR) ovf = true;  // support too large
-          if (want && !ovf && cnt > 0) {
-            // stored values are compared in stored units; a key a rounding
-            // step below the bound is harmless (the exact solve drops it)
+          // append the candidates: the chunk goes to a per-thread stash so
+          // that the loop runs once per candidate, not once per key.  Stored
+          // values are compared in stored units; a key a rounding step below
+          // the bound is harmless (the exact solve drops it).
+          if (__any_sync(0xffffffffu, msk != 0)) {
+            float stash[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) stash[k] = __uint_as_float(rc[k]);
             int2* ptr = mybuf + nbuf;
             const int kj = j0 + c * 32;
-            float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              const float v = __uint_as_float(r[c * 32 + k]);
-              if (v > thr) {
-                *ptr = make_int2(kj + k, __float_as_int(v));
-                ++ptr;
-                if (k & 1) s1 += v; else s0 += v;
-              }
+            float sadd = 0.f;
+            while (msk) {
+              const int k = __ffs(msk) - 1;
+              msk &= msk - 1;
+              const float v = stash[k];
+              *ptr++ = make_int2(kj + k, __float_as_int(v));
+              sadd += v;
             }
             nbuf += cnt;
-            bsum += s0 + s1;
+            bsum += sadd;
           }
         }
       }
@@ -631,76 +595,25 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
 
     // ---- epilogue ----------------------------------------------------------
     if constexpr (MODE == TC_TAU) {
-      // exact tau and the support list of every row, one row at a time with
-      // the whole warp; with split rows the two halves' buffers are merged
-      // (each half's bound is a valid bound of the whole row's threshold)
-      float4* xs = reinterpret_cast<float4*>(smem + LY::OFF_Q);  // Q is no longer read
-      if constexpr (NH > 1) {
-        xs[half * TC_BM + row] = make_float4(m_run, lb, __int_as_float(nbuf), ovf ? 1.f : 0.f);
-        asm volatile("bar.sync 1, %0;" ::"r"(NWN * 32) : "memory");
-      } else {
-        __syncwarp();
-      }
-      constexpr int RPW = 32 / NH;  // rows this warp finishes
+      // exact tau and the support list of every row, each thread its own
       const float vs = fast ? zs : 1.f;
-      for (int i = 0; i < RPW; ++i) {
-        const int rloc = half * RPW + i;          // row within the quarter
-        const int rq = quarter * 32 + rloc;       // row within the tile
-        const int qr = q0 + rq;
-        if (qr >= P.Tq) break;
-        const size_t fr = (size_t)bh * P.Tq + qr;
-        float m_r, lb_r;
-        int n0, n1 = 0;
-        bool ovf_r;
-        if constexpr (NH > 1) {
-          const float4 a0 = xs[rq], a1 = xs[TC_BM + rq];
-          m_r = fmaxf(a0.x, a1.x);
-          lb_r = fmaxf(a0.y, a1.y);
-          n0 = __float_as_int(a0.z);
-          n1 = __float_as_int(a1.z);
-          ovf_r = a0.w != 0.f || a1.w != 0.f;
-        } else {
-          m_r = __shfl_sync(0xffffffffu, m_run, rloc);
-          lb_r = __shfl_sync(0xffffffffu, lb, rloc);
-          n0 = __shfl_sync(0xffffffffu, nbuf, rloc);
-          ovf_r = __shfl_sync(0xffffffffu, (int)ovf, rloc) != 0;
-        }
+      if (row_ok) {
         float t = INFINITY;
         int nsup = 0;
-        if (ovf_r) {
-          if (lane == 0) {
-            const int slot = atomicAdd(A.ovf_count, 1);
-            A.ovf_rows[slot] = (int)fr;
-          }
-        } else if (m_r != -INFINITY) {
-          const int2* b0 = bufbase + (size_t)rq * LY::CAP_STRIDE;
-          const int2* b1 = bufbase + (size_t)(TC_BM + rq) * LY::CAP_STRIDE;
-          RowEntries ent;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int k = lane + 32 * e;
-            ent.e[e] = (k < n0) ? b0[k]
-                       : (k < n0 + n1) ? b1[k - n0]
-                                       : make_int2(0, __float_as_int(-INFINITY));
-          }
-          t = warp_row_tau(ent, vs, m_r, entmax, lb_r - m_r);
-          int2* dst = A.sup_list + fr * (size_t)A.sup_cap;
-          const unsigned below = (1u << lane) - 1u;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float x = __int_as_float(ent.e[e].y) * vs - t;
-            const bool in = x > 0.f;
-            const unsigned bal = __ballot_sync(0xffffffffu, in);
-            if (in)
-              dst[nsup + __popc(bal & below)] =
-                  make_int2(ent.e[e].x, __float_as_int(entmax ? x * x : x));
-            nsup += __popc(bal);
+        if (ovf) {
+          const int slot = atomicAdd(A.ovf_count, 1);
+          A.ovf_rows[slot] = (int)flat;
+        } else if (m_run != -INFINITY) {
+          t = thread_row_tau(mybuf, nbuf, vs, m_run, entmax, lb - m_run);
+          int2* dst = A.sup_list + flat * (size_t)A.sup_cap;
+          for (int i = 0; i < nbuf; ++i) {
+            const int2 e = mybuf[i];
+            const float x = __int_as_float(e.y) * vs - t;
+            if (x > 0.f) dst[nsup++] = make_int2(e.x, __float_as_int(entmax ? x * x : x));
           }
         }
-        if (lane == 0) {
-          A.tau[fr] = t;
-          A.sup_count[fr] = nsup;
-        }
+        A.tau[flat] = t;
+        A.sup_count[flat] = nsup;
       }
     } else {
       const bool have_o =
