@@ -176,7 +176,10 @@ LAUNCHES = {"softmax": 1, "softmax1": 1, "sparsemax": 3, "entmax15": 3}
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
 # capture of the current kernel (the profile summary named beside it).
 # An entry is removed whenever the kernel changes after its capture.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    ("qwen3_8b_prefill", "softmax"): (
+        132_658_176, "profiles/prefill_pair_qwen3_8b_softmax.md"),
+}
 LAUNCHES_DECODE = {"softmax": 2, "softmax1": 2, "sparsemax": 4, "entmax15": 4}
 
 
