@@ -327,9 +327,10 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
   A.sup_cap = pl.sup_cap;
   if (cudaMemsetAsync(A.ovf_count, 0, sizeof(int), st) != cudaSuccess) return NATTN_ECUDA;
   {
-    // whole rows per thread: splitting rows halves each buffer, and the
-    // larger buffers measured faster for the wider 1.5-entmax supports
-    constexpr int NHT = 1;
+    // d <= 128: each S row split between two warps (eight normalizer warps
+    // hide each other's latency; the halves share their bounds); d = 256
+    // keeps whole rows (64-key blocks leave 32 columns per half)
+    constexpr int NHT = (D <= 128) ? 2 : 1;
     using LY = TcLayout<D, D, BN, 2, 1, TC_TAU, NHT>;
     auto k = prefill_tc_kernel<D, D, BN, 2, 1, TC_TAU, NHT>;
     if (allow_smem(k, LY::ALLOC) != cudaSuccess) return NATTN_ECUDA;

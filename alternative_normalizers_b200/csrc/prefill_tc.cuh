@@ -72,7 +72,7 @@ struct TcArgs {
 // thread holds half a row in registers.
 template <int D, int DV, int BN, int KST, int VST, int MODE, int NH = 1>
 struct TcLayout {
-  static_assert(NH == 1 || MODE == TC_ONLINE, "row split is for the online mode");
+  static_assert(NH == 1 || MODE != TC_APPLY, "row split is for the online and tau modes");
   static constexpr int NWN = 4 * NH;                 // normalizer warps
   static constexpr int THREADS = (NWN + 2) * 32;     // + TMA warp + MMA warp
   static constexpr int QBYTES = D * TC_BM * 2;
@@ -86,8 +86,15 @@ struct TcLayout {
   static constexpr int CAPR = CAP / NH;         // entries per row half
   static constexpr int CAP_STRIDE = CAPR + 1;    // int2 entries per row half
   static constexpr int BUFBYTES = (MODE == TC_TAU) ? CAP_STRIDE * TC_BM * NH * 8 : 0;
-  static constexpr int OFF_BAR = OFF_BUF + BUFBYTES;
-  static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 2 + 2 + 1;
+  // split rows in the threshold pass: each half publishes its running lower
+  // bound of the row's threshold for the other half
+  static constexpr int LBXBYTES = (MODE == TC_TAU && NH > 1) ? NH * TC_BM * 4 : 0;
+  static constexpr int OFF_LBX = OFF_BUF + BUFBYTES;
+  static constexpr int OFF_BAR = OFF_LBX + LBXBYTES;
+  // S ring depth in TMEM: the threshold pass has no O accumulator, so it
+  // keeps four S buffers and its normalizer warps can drift three blocks apart
+  static constexpr int NSB = (MODE == TC_TAU) ? 4 : 2;
+  static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 2 * NSB + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // epilogue (m, l) exchange between row halves: reuses the Q tile, which
   // every product has finished reading once the last PV has completed
@@ -95,10 +102,9 @@ struct TcLayout {
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
   // TMEM columns: S double buffer, then O
-  static constexpr int TM_S0 = 0;
-  static constexpr int TM_S1 = BN;
+  static constexpr int TM_S = 0;  // S buffer s at column s * BN
   static constexpr int TM_O = 2 * BN;
-  static constexpr int TM_COLS_USED = (MODE == TC_TAU) ? 2 * BN : 2 * BN + NH * DV;
+  static constexpr int TM_COLS_USED = (MODE == TC_TAU) ? NSB * BN : 2 * BN + NH * DV;
   static constexpr int TM_COLS = TM_COLS_USED <= 32    ? 32
                                  : TM_COLS_USED <= 64  ? 64
                                  : TM_COLS_USED <= 128 ? 128
@@ -127,21 +133,26 @@ __device__ __forceinline__ float tc_z(float s, const TcArgs& A) {
 // first and accepted once it satisfies the optimality conditions (all members
 // above it, everything else at or below it); for sparsemax this is Michelot's
 // projection algorithm.
-__device__ __forceinline__ float thread_row_tau(const int2* row, int n, float vscale, float m,
-                                                bool entmax, float t0) {
+__device__ __forceinline__ float thread_row_tau(const int2* row0, int n0, const int2* row1,
+                                                int n1, float vscale, float m, bool entmax,
+                                                float t0) {
   float t = fmaxf(t0, -1.f);
   for (int it = 0; it < 64; ++it) {
     float cnt = 0.f, s1 = 0.f, s2 = 0.f, wmin = INFINITY;
+    auto add = [&](const int2* row, int n) {
 #pragma unroll 4
-    for (int i = 0; i < n; ++i) {
-      const float w = __int_as_float(row[i].y) * vscale - m;
-      if (w > t) {
-        cnt += 1.f;
-        s1 += w;
-        s2 = fmaf(w, w, s2);
-        wmin = fminf(wmin, w);
+      for (int i = 0; i < n; ++i) {
+        const float w = __int_as_float(row[i].y) * vscale - m;
+        if (w > t) {
+          cnt += 1.f;
+          s1 += w;
+          s2 = fmaf(w, w, s2);
+          wmin = fminf(wmin, w);
+        }
       }
-    }
+    };
+    add(row0, n0);
+    add(row1, n1);
     float ts, tn;
     bool valid = true;
     if (!entmax) {
@@ -190,6 +201,7 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
   using LY = TcLayout<D, DV, BN, KST, VST, MODE, NH>;
   constexpr int NWN = LY::NWN;
   constexpr int NC = BN / NH;  // S columns per normalizer thread
+  constexpr int NSB = LY::NSB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -220,11 +232,15 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
   auto bar_vfull = [&](int s) { return smem_addr(&bars[1 + 2 * KST + s]); };
   auto bar_vempty = [&](int s) { return smem_addr(&bars[1 + 2 * KST + VST + s]); };
   auto bar_sfull = [&](int s) { return smem_addr(&bars[1 + 2 * KST + 2 * VST + s]); };
-  auto bar_pfull = [&](int s) { return smem_addr(&bars[1 + 2 * KST + 2 * VST + 2 + s]); };
-  const uint32_t bar_pv = smem_addr(&bars[1 + 2 * KST + 2 * VST + 4]);
+  auto bar_pfull = [&](int s) { return smem_addr(&bars[1 + 2 * KST + 2 * VST + NSB + s]); };
+  const uint32_t bar_pv = smem_addr(&bars[1 + 2 * KST + 2 * VST + 2 * NSB]);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + LY::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
 
+  if constexpr (LY::LBXBYTES > 0) {
+    float* lbx = reinterpret_cast<float*>(smem + LY::OFF_LBX);
+    for (int i = tid; i < NH * TC_BM; i += LY::THREADS) lbx[i] = -INFINITY;
+  }
   if (tid == 0) {
     mbar_init(bar_q, 1);
     for (int s = 0; s < KST; ++s) {
@@ -235,7 +251,7 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
       mbar_init(bar_vfull(s), 1);
       mbar_init(bar_vempty(s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NSB; ++s) {
       mbar_init(bar_sfull(s), 1);
       mbar_init(bar_pfull(s), NWN);
     }
@@ -296,7 +312,7 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
       tc_fence_after();
       for (int j = 0; ok && j <= nblk; ++j) {
         if (j < nblk) {
-          const int sb = j & 1, ks = j % KST;
+          const int sb = j % NSB, ks = j % KST;
           if (!mbar_wait_spin(bar_kfull(ks), (j / KST) & 1, abort_flag)) break;
           // S buffer sb held P_{j-2}.  With a PV product that reads it, that
           // product was issued by this thread before this QK and tcgen05.mma
@@ -304,12 +320,12 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
           // needed; without one (threshold pass) the normalizer warps must be
           // done reading S_{j-2}.
           if constexpr (MODE == TC_TAU) {
-            if (j >= 2 && !mbar_wait_spin(bar_pfull(sb), ((j - 2) / 2) & 1, abort_flag))
+            if (j >= NSB && !mbar_wait_spin(bar_pfull(sb), ((j - NSB) / NSB) & 1, abort_flag))
               break;
           }
           tc_fence_after();
           const uint32_t kbase = smem_addr(smem + LY::OFF_K + ks * LY::KBYTES);
-          const uint32_t sdst = tmem + (sb ? LY::TM_S1 : LY::TM_S0);
+          const uint32_t sdst = tmem + LY::TM_S + sb * BN;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t ad =
@@ -323,12 +339,12 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
         }
         if constexpr (MODE != TC_TAU) {
           if (j >= 1) {
-            const int jp = j - 1, sbp = jp & 1, vs = jp % VST;
-            if (!mbar_wait_spin(bar_pfull(sbp), (jp / 2) & 1, abort_flag)) break;
+            const int jp = j - 1, sbp = jp % NSB, vs = jp % VST;
+            if (!mbar_wait_spin(bar_pfull(sbp), (jp / NSB) & 1, abort_flag)) break;
             if (!mbar_wait_spin(bar_vfull(vs), (jp / VST) & 1, abort_flag)) break;
             tc_fence_after();
             const uint32_t vbase = smem_addr(smem + LY::OFF_V + vs * LY::VBYTES);
-            const uint32_t pt = tmem + (sbp ? LY::TM_S1 : LY::TM_S0);
+            const uint32_t pt = tmem + LY::TM_S + sbp * BN;
 #pragma unroll
             for (int hh = 0; hh < NH; ++hh) {
               // half hh: its packed P sits at the start of its own S columns,
@@ -371,6 +387,9 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
     float m_run, l_run = 0.f, tau = 0.f;
     // TAU state
     int2* const bufbase = reinterpret_cast<int2*>(smem + LY::OFF_BUF);
+    volatile float* const lbx_mine = reinterpret_cast<float*>(smem + LY::OFF_LBX) + half * TC_BM + row;
+    volatile float* const lbx_other =
+        reinterpret_cast<float*>(smem + LY::OFF_LBX) + (NH - 1 - half) * TC_BM + row;
     int2* tbuf = bufbase + (size_t)(half * TC_BM + quarter * 32) * LY::CAP_STRIDE;  // 32 rows
     int2* mybuf = tbuf + lane * LY::CAP_STRIDE;
     int nbuf = 0;
@@ -390,8 +409,8 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
     bool alive = true;
 
     for (int j = 0; j < nblk; ++j) {
-      const int sb = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait_spin(bar_sfull(sb), (j / 2) & 1, abort_flag))) {
+      const int sb = j % NSB;
+      if (!__all_sync(0xffffffffu, mbar_wait_spin(bar_sfull(sb), (j / NSB) & 1, abort_flag))) {
         alive = false;
         break;
       }
@@ -405,10 +424,10 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
         klb = NC;
         span = 0;
       }
-      const uint32_t sbase = lane_base + (sb ? LY::TM_S1 : LY::TM_S0) + cbase;
+      const uint32_t sbase = lane_base + LY::TM_S + sb * BN + cbase;
       // the online mode needs its whole part of the row at once (maximum
       // before exponentials); the sparse modes work on 64-key sub-blocks
-      constexpr int LDC = (MODE == TC_ONLINE) ? NC : 64;
+      constexpr int LDC = (MODE == TC_ONLINE || NC < 64) ? NC : 64;
 #pragma unroll 1
       for (int hs = 0; hs < NC / LDC; ++hs) {
       const uint32_t saddr = sbase + hs * LDC;       // S columns of this sub-block
@@ -526,6 +545,12 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
             const float su = bsum * vs;
             lb = fmaxf(lb, entmax ? __fdividef(su, fn) - rsqrtf(fn) : __fdividef(su - 1.f, fn));
           }
+          if constexpr (NH > 1) {
+            // a bound of one half's keys bounds the whole row; a stale read
+            // of the other half's value is still a valid bound
+            lb = fmaxf(lb, lbx_other[0]);
+            lbx_mine[0] = lb;
+          }
           const bool want = cmax > lb && !ovf;
           if (!__any_sync(0xffffffffu, want)) continue;
           // candidates are tested in stored units against the bound less a
@@ -545,45 +570,57 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
             return mk;
           };
           unsigned msk = want ? cand_mask(thr) : 0u;
-          int cnt = __popc(msk);
-          // when a row's buffer cannot take this chunk's candidates, every row
-          // of the warp raises its bound to the exact threshold of the keys
-          // it has seen and compacts (each thread its own row, side by side:
-          // the rows of a tile fill their buffers at similar rates, so one
-          // batch stands in for many single-row solves)
-          if (__any_sync(0xffffffffu, nbuf + cnt > LY::CAPR)) {
-            lb = fmaxf(lb, thread_row_tau(mybuf, nbuf, vs, m_run, entmax, lb - m_run));
-            nbuf = thread_compact_row(mybuf, nbuf, vs, lb, &bsum);
-            thr = to_thr(lb);
-            msk = want ? cand_mask(thr) : 0u;
-            cnt = __popc(msk);
-            if (nbuf + cnt > LY::CAPR) {  // support too large for the buffer
-              ovf = true;
-              msk = 0;
-              cnt = 0;
-            }
-          }
-          // append the candidates: the chunk goes to a per-thread stash so
-          // that the loop runs once per candidate, not once per key.  Stored
-          // values are compared in stored units; a key a rounding step below
-          // the bound is harmless (the exact solve drops it).
-          if (__any_sync(0xffffffffu, msk != 0)) {
-            float stash[32];
+          // the chunk goes to a per-thread stash so that appends run once per
+          // candidate, not once per key
+          float stash[32];
 #pragma unroll
-            for (int k = 0; k < 32; ++k) stash[k] = __uint_as_float(rc[k]);
+          for (int k = 0; k < 32; ++k) stash[k] = __uint_as_float(rc[k]);
+          const int kj = j0 + c * 32;
+          // append candidates (lowest key first) while there is room; stored
+          // values are compared in stored units, and a key a rounding step
+          // below the bound is harmless (the exact solve drops it)
+          auto append = [&](int room) {
             int2* ptr = mybuf + nbuf;
-            const int kj = j0 + c * 32;
             float sadd = 0.f;
-            while (msk) {
+            int na = 0;
+            while (msk && na < room) {
               const int k = __ffs(msk) - 1;
               msk &= msk - 1;
               const float v = stash[k];
               *ptr++ = make_int2(kj + k, __float_as_int(v));
               sadd += v;
+              ++na;
             }
-            nbuf += cnt;
+            nbuf += na;
             bsum += sadd;
+          };
+          // when a row's buffer cannot take this chunk's candidates, every row
+          // of the warp raises its bound to the exact threshold of the keys
+          // it has seen and compacts (each thread its own row, side by side:
+          // the rows of a tile fill their buffers at similar rates, so one
+          // batch stands in for many single-row solves)
+          if (__any_sync(0xffffffffu, nbuf + __popc(msk) > LY::CAPR)) {
+            lb = fmaxf(lb, thread_row_tau(mybuf, nbuf, mybuf, 0, vs, m_run, entmax, lb - m_run));
+            nbuf = thread_compact_row(mybuf, nbuf, vs, lb, &bsum);
+            thr = to_thr(lb);
+            msk &= cand_mask(thr);
+            // still too many: take candidates until the buffer is full and
+            // solve again with them included (they are seen keys too), a few
+            // rounds at most; a row that still cannot fit goes to the
+            // row-wise pass
+            for (int round = 0; round < 4 && nbuf + __popc(msk) > LY::CAPR; ++round) {
+              append(LY::CAPR - nbuf);
+              lb = fmaxf(lb, thread_row_tau(mybuf, nbuf, mybuf, 0, vs, m_run, entmax, lb - m_run));
+              nbuf = thread_compact_row(mybuf, nbuf, vs, lb, &bsum);
+              msk &= cand_mask(to_thr(lb));
+            }
+            if (nbuf + __popc(msk) > LY::CAPR) {
+              ovf = true;
+              msk = 0;
+            }
+            if constexpr (NH > 1) lbx_mine[0] = lb;
           }
+          if (__any_sync(0xffffffffu, msk != 0)) append(32);
         }
       }
       }  // sub-blocks
@@ -595,22 +632,48 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
 
     // ---- epilogue ----------------------------------------------------------
     if constexpr (MODE == TC_TAU) {
-      // exact tau and the support list of every row, each thread its own
+      // exact tau and the support list of every row, one thread per row;
+      // with split rows the two halves' buffers are merged (each half's
+      // bound is a valid bound of the whole row's threshold) and the row's
+      // two warps take one half of the quarter's rows each
       const float vs = fast ? zs : 1.f;
-      if (row_ok) {
+      float m_r = m_run, lb_r = lb;
+      int n0 = nbuf, n1 = 0;
+      bool ovf_r = ovf, mine = true;
+      const int2* b0 = mybuf;
+      const int2* b1 = mybuf;
+      if constexpr (NH > 1) {
+        float4* xs = reinterpret_cast<float4*>(smem + LY::OFF_Q);  // Q is no longer read
+        xs[half * TC_BM + row] = make_float4(m_run, lb, __int_as_float(nbuf), ovf ? 1.f : 0.f);
+        asm volatile("bar.sync 1, %0;" ::"r"(NWN * 32) : "memory");
+        const float4 a0 = xs[row], a1 = xs[TC_BM + row];
+        m_r = fmaxf(a0.x, a1.x);
+        lb_r = fmaxf(a0.y, a1.y);
+        n0 = __float_as_int(a0.z);
+        n1 = __float_as_int(a1.z);
+        ovf_r = a0.w != 0.f || a1.w != 0.f;
+        b0 = bufbase + (size_t)row * LY::CAP_STRIDE;
+        b1 = bufbase + (size_t)(TC_BM + row) * LY::CAP_STRIDE;
+        mine = (lane >> 4) == half;
+      }
+      if (row_ok && mine) {
         float t = INFINITY;
         int nsup = 0;
-        if (ovf) {
+        if (ovf_r) {
           const int slot = atomicAdd(A.ovf_count, 1);
           A.ovf_rows[slot] = (int)flat;
-        } else if (m_run != -INFINITY) {
-          t = thread_row_tau(mybuf, nbuf, vs, m_run, entmax, lb - m_run);
+        } else if (m_r != -INFINITY) {
+          t = thread_row_tau(b0, n0, b1, n1, vs, m_r, entmax, lb_r - m_r);
           int2* dst = A.sup_list + flat * (size_t)A.sup_cap;
-          for (int i = 0; i < nbuf; ++i) {
-            const int2 e = mybuf[i];
-            const float x = __int_as_float(e.y) * vs - t;
-            if (x > 0.f) dst[nsup++] = make_int2(e.x, __float_as_int(entmax ? x * x : x));
-          }
+          auto emit = [&](const int2* src, int n) {
+            for (int i = 0; i < n; ++i) {
+              const int2 e = src[i];
+              const float x = __int_as_float(e.y) * vs - t;
+              if (x > 0.f) dst[nsup++] = make_int2(e.x, __float_as_int(entmax ? x * x : x));
+            }
+          };
+          emit(b0, n0);
+          emit(b1, n1);
         }
         A.tau[flat] = t;
         A.sup_count[flat] = nsup;
