@@ -266,7 +266,7 @@ int check_launch() {
 int launch_rowwise(const Problem& P, const Plan& pl, const int* row_list,
                    const int* row_count, int nrows, float* slots, int grid,
                    cudaStream_t st) {
-  const int bytes = (256 + 64 + ROW_THREADS + pl.row_cap) * 4;
+  const int bytes = (256 + 64 + ROW_WARPS * 256 + pl.row_cap) * 4;
   if (allow_smem(rowwise_kernel, bytes) != cudaSuccess) return NATTN_ECUDA;
   rowwise_kernel<<<grid, ROW_THREADS, bytes, st>>>(P, row_list, row_count, nrows,
                                                    pl.row_cap, slots);

@@ -121,17 +121,18 @@ __device__ float block_solve_tau(const float* sc, int n, float m, bool entmax,
 }
 
 // One CTA per query row (grid-stride over rows).  Dynamic shared memory:
-// q as float [256] | reduction scratch [64] | column partials [256] |
-// scores [cap].
+// q as float [256] | reduction scratch [64] | column partials
+// [ROW_WARPS * 256] | scores [cap].
 __global__ void __launch_bounds__(ROW_THREADS)
     rowwise_kernel(Problem P, const int* __restrict__ row_list,
                    const int* __restrict__ row_count, int nrows_static, int cap,
                    float* __restrict__ gslots) {
   extern __shared__ float smem_f[];
+  __shared__ int s_ncand;
   float* qf = smem_f;
   float* red = qf + 256;
   float* part = red + 64;
-  float* sc_smem = part + ROW_THREADS;
+  float* sc_smem = part + ROW_WARPS * 256;
   const int tid = threadIdx.x;
   const int nrows = row_count ? *row_count : nrows_static;
   const int group = P.Hq / P.Hkv;
@@ -165,29 +166,64 @@ __global__ void __launch_bounds__(ROW_THREADS)
       qf[c] = __bfloat162float(P.q[(size_t)flat * P.d + c]);
     __syncthreads();
 
-    // scores z_j for the allowed keys, in units fixed by the normalizer
+    // scores z_j for the allowed keys, in units fixed by the normalizer.
+    // Eight lanes share one key row (16-byte loads, coalesced), four keys
+    // per warp and KU keys per lane group in flight.
     const float uscale = (P.norm == NATTN_ENTMAX15) ? 0.5f : 1.0f;
     int badkey = 0;
-    for (int jj = tid; jj < n; jj += ROW_THREADS) {
-      const int j = rr.lo + jj;
-      bool kb = false;
-      const bf16* kp = key_row(P, P.k, P.d, b, g, j, kb);
-      float s = 0.f;
-      if (!kb) {
-        const uint4* k4 = reinterpret_cast<const uint4*>(kp);
-        for (int c8 = 0; c8 < P.d / 8; ++c8) {
-          const uint4 x = k4[c8];
-          const float* qq = qf + c8 * 8;
-          s += qq[0] * bf16lo(x.x) + qq[1] * bf16hi(x.x) + qq[2] * bf16lo(x.y) +
-               qq[3] * bf16hi(x.y) + qq[4] * bf16lo(x.z) + qq[5] * bf16hi(x.z) +
-               qq[6] * bf16lo(x.w) + qq[7] * bf16hi(x.w);
+    {
+      constexpr int KU = 4;
+      constexpr int STEP = ROW_WARPS * 4;  // keys per pass of all warps
+      const int lane = tid & 31, sub = lane & 7;
+      const int nc8 = P.d / 8;  // 16-byte chunks per key row (at most 32)
+      // the loop bound is the warp's first key, so every lane of a warp runs
+      // the same iterations (the shuffles below need all 32 lanes)
+      for (int wb = (tid >> 5) * 4; wb < n; wb += STEP * KU) {
+        const int base = wb + (lane >> 3);
+        uint4 x[KU][4];
+#pragma unroll
+        for (int u = 0; u < KU; ++u) {
+          const int jj = base + u * STEP;
+          bool kb = false;
+          const uint4* k4 = nullptr;
+          if (jj < n) {
+            k4 = reinterpret_cast<const uint4*>(key_row(P, P.k, P.d, b, g, rr.lo + jj, kb));
+            if (kb) {
+              badkey = 1;
+              k4 = nullptr;
+            }
+          }
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int c8 = sub + 8 * t;
+            x[u][t] = (k4 != nullptr && c8 < nc8) ? k4[c8] : make_uint4(0u, 0u, 0u, 0u);
+          }
         }
-      } else {
-        badkey = 1;
+#pragma unroll
+        for (int u = 0; u < KU; ++u) {
+          float s = 0.f;
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int c8 = sub + 8 * t;
+            if (c8 < nc8) {
+              const float* qq = qf + c8 * 8;
+              const uint4 y = x[u][t];
+              s += qq[0] * bf16lo(y.x) + qq[1] * bf16hi(y.x) + qq[2] * bf16lo(y.y) +
+                   qq[3] * bf16hi(y.y) + qq[4] * bf16lo(y.z) + qq[5] * bf16hi(y.z) +
+                   qq[6] * bf16lo(y.w) + qq[7] * bf16hi(y.w);
+            }
+          }
+          s += __shfl_xor_sync(0xffffffffu, s, 1);
+          s += __shfl_xor_sync(0xffffffffu, s, 2);
+          s += __shfl_xor_sync(0xffffffffu, s, 4);
+          const int jj = base + u * STEP;
+          if (sub == 0 && jj < n) {
+            float z = s * P.scale;
+            if (P.softcap > 0.f) z = P.softcap * tanhf(z / P.softcap);
+            sc[jj] = z * uscale;
+          }
+        }
       }
-      float z = s * P.scale;
-      if (P.softcap > 0.f) z = P.softcap * tanhf(z / P.softcap);
-      sc[jj] = z * uscale;
     }
     if (__syncthreads_or(badkey)) bad = true;
     if (bad) {
@@ -219,8 +255,27 @@ __global__ void __launch_bounds__(ROW_THREADS)
       float mx = -INFINITY;
       for (int jj = tid; jj < n; jj += ROW_THREADS) mx = fmaxf(mx, sc[jj]);
       mx = block_max(mx, red);
+      // the threshold is at least max - 1 (in threshold units), so the solve
+      // runs over the keys within one unit of the maximum, gathered into the
+      // column-partials area (free until the PV), unless there are too many
       float tau = INFINITY;
-      if (n > 0) tau = block_solve_tau(sc, n, mx, ent, red);
+      if (n > 0) {
+        float* cand = part;
+        constexpr int kCandCap = ROW_WARPS * 256;
+        if (tid == 0) s_ncand = 0;
+        __syncthreads();
+        for (int jj = tid; jj < n; jj += ROW_THREADS) {
+          const float u = sc[jj];
+          if (u > mx - 1.f) {
+            const int k = atomicAdd(&s_ncand, 1);
+            if (k < kCandCap) cand[k] = u;
+          }
+        }
+        __syncthreads();
+        const int nc = s_ncand;
+        tau = (nc <= kCandCap) ? block_solve_tau(cand, nc, mx, ent, red)
+                               : block_solve_tau(sc, n, mx, ent, red);
+      }
       __syncthreads();
       for (int jj = tid; jj < n; jj += ROW_THREADS) {
         const float t = fmaxf(sc[jj] - tau, 0.f);
@@ -238,27 +293,68 @@ __global__ void __launch_bounds__(ROW_THREADS)
       }
     }
 
-    // O = p V: thread (grp, c) sums keys grp, grp + G, ... for column c
-    const int G = ROW_THREADS / P.dv;
-    const int c = tid % P.dv, grp = tid / P.dv;
-    float acc = 0.f;
-    if (grp < G) {
-      for (int jj = grp; jj < n; jj += G) {
-        const float p = sc[jj];
-        if (p != 0.f) {
-          bool kb = false;
-          const bf16* vp = key_row(P, P.v, P.dv, b, g, rr.lo + jj, kb);
-          acc += p * __bfloat162float(vp[c]);
+    if (P.norm == NATTN_SOFTMAX || P.norm == NATTN_SOFTMAX1) {
+      // O = p V: thread (grp, c) sums keys grp, grp + G, ... for column c
+      const int G = ROW_THREADS / P.dv;
+      const int c = tid % P.dv, grp = tid / P.dv;
+      float acc = 0.f;
+      if (grp < G) {
+        for (int jj = grp; jj < n; jj += G) {
+          const float p = sc[jj];
+          if (p != 0.f) {
+            bool kb = false;
+            const bf16* vp = key_row(P, P.v, P.dv, b, g, rr.lo + jj, kb);
+            acc += p * __bfloat162float(vp[c]);
+          }
         }
       }
-    }
-    __syncthreads();
-    if (grp < G) part[grp * P.dv + c] = acc;
-    __syncthreads();
-    if (tid < P.dv) {
-      float o = 0.f;
-      for (int q2 = 0; q2 < G; ++q2) o += part[q2 * P.dv + tid];
-      orow[tid] = __float2bfloat16_rn(o);
+      __syncthreads();
+      if (grp < G) part[grp * P.dv + c] = acc;
+      __syncthreads();
+      if (tid < P.dv) {
+        float o = 0.f;
+        for (int q2 = 0; q2 < G; ++q2) o += part[q2 * P.dv + tid];
+        orow[tid] = __float2bfloat16_rn(o);
+      }
+    } else {
+      // sparse weights: each warp scans its slice of the keys 32 at a time
+      // and, for every nonzero weight a ballot finds, adds the whole V row
+      // (lane c holds columns c, c + 32, ...); the warps' sums are then added
+      const int lane = tid & 31, wrp = tid >> 5;
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      const int per = (n + ROW_WARPS - 1) / ROW_WARPS;
+      const int j0 = wrp * per, j1 = min(n, j0 + per);
+      for (int jb = j0; jb < j1; jb += 32) {
+        const int jj = jb + lane;
+        const float p = (jj < j1) ? sc[jj] : 0.f;
+        unsigned nz = __ballot_sync(0xffffffffu, p != 0.f);
+        while (nz) {
+          const int src = __ffs(nz) - 1;
+          nz &= nz - 1;
+          const float pj = __shfl_sync(0xffffffffu, p, src);
+          bool kb = false;
+          const bf16* vp = key_row(P, P.v, P.dv, b, g, rr.lo + jb + src, kb);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int c = lane + 32 * i;
+            if (c < P.dv) acc[i] += pj * __bfloat162float(vp[c]);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = lane + 32 * i;
+        if (c < P.dv) part[wrp * 256 + c] = acc[i];
+      }
+      __syncthreads();
+      if (tid < P.dv) {
+        float o = 0.f;
+#pragma unroll
+        for (int w = 0; w < ROW_WARPS; ++w) o += part[w * 256 + tid];
+        orow[tid] = __float2bfloat16_rn(o);
+      }
     }
     if (tid == 0 && P.row_stat) P.row_stat[flat] = stat;
     __syncthreads();
