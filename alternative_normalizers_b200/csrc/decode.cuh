@@ -45,6 +45,10 @@ struct DecodeArgs {
   float* ml;      // [B*Hkv*nsplit*R][2]      (ONLINE: m, l; SCORES: max)
   float* scores;  // [B*Hq*Tq][Tk]            (SCORES / APPLY)
   const float* tau;  // [B*Hq*Tq]             (APPLY)
+  // pages of each row holding a nonzero weight, one bit per page, written by
+  // the threshold kernel and read by APPLY: [B*Hq*Tq][pm_words]
+  unsigned* pmask;
+  int pm_words;
 };
 
 constexpr int DEC_THREADS = 128;
@@ -128,20 +132,17 @@ __global__ void __launch_bounds__(DEC_THREADS)
   // ---- APPLY: which pages of this split carry any nonzero weight ----------
   int count = p_end - p_begin;
   if constexpr (MODE == DEC_APPLY) {
+    // a page is loaded when any row of the group has a nonzero weight in it
+    // (bits set by the threshold kernel)
     int* pflag = plist + A.pps;
-    for (int p = p_begin + warp; p < p_end; p += DEC_THREADS / 32) {
-      int any = 0;
+    for (int p = p_begin + tid; p < p_end; p += DEC_THREADS) {
+      unsigned any = 0;
       for (int r = 0; r < R; ++r) {
         const int hh = r / P.Tq, i = r % P.Tq;
         const size_t row = ((size_t)b * P.Hq + g * group + hh) * P.Tq + i;
-        const float tr = A.tau[row];
-        for (int jj = lane; jj < PS; jj += 32) {
-          const int j = p * PS + jj;
-          if (j < Lk && A.scores[row * P.Tk + j] > tr) any = 1;
-        }
+        any |= (A.pmask[row * A.pm_words + (p >> 5)] >> (p & 31)) & 1u;
       }
-      any = __any_sync(0xffffffffu, any);
-      if (lane == 0) pflag[p - p_begin] = any;
+      pflag[p - p_begin] = (int)any;
     }
     __syncthreads();
     if (tid == 0) {  // compact in page order so the sums are deterministic
@@ -488,7 +489,9 @@ __global__ void __launch_bounds__(TAU_THREADS)
     decode_tau_kernel(DecodeArgs A, float* tau_out, int cap) {
   extern __shared__ float tsm[];
   float* red = tsm;
-  float* cand = tsm + 64;
+  float* cand = tsm + 64;                                     // [cap] values
+  int* cidx = reinterpret_cast<int*>(cand + cap);             // [cap] key indices
+  unsigned* smask = reinterpret_cast<unsigned*>(cidx + cap);  // [pm_words]
   __shared__ int s_n;
   const Problem& P = A.P;
   const int row = blockIdx.x;
@@ -499,8 +502,10 @@ __global__ void __launch_bounds__(TAU_THREADS)
   const int g = h / group, r = (h % group) * P.Tq + i;
   const int Lk = P.seqlens[b];
   const bool valid = !(Lk < 1 || Lk > P.Tk || Lk > P.bt_stride * P.page_size);
+  unsigned* prow = A.pmask + (size_t)row * A.pm_words;
   if (!valid) {
     if (threadIdx.x == 0) tau_out[row] = INFINITY;
+    for (int w = threadIdx.x; w < A.pm_words; w += TAU_THREADS) prow[w] = 0u;
     return;
   }
   const int npages = (Lk + P.page_size - 1) / P.page_size;
@@ -510,16 +515,21 @@ __global__ void __launch_bounds__(TAU_THREADS)
   for (int s = 0; s < nact; ++s) m = fmaxf(m, A.ml[(pbase + (size_t)s * A.R) * 2]);
   if (m == -INFINITY) {  // no visible key
     if (threadIdx.x == 0) tau_out[row] = INFINITY;
+    for (int w = threadIdx.x; w < A.pm_words; w += TAU_THREADS) prow[w] = 0u;
     return;
   }
   if (threadIdx.x == 0) s_n = 0;
+  for (int w = threadIdx.x; w < A.pm_words; w += TAU_THREADS) smask[w] = 0u;
   __syncthreads();
   const float* zrow = A.scores + (size_t)row * P.Tk;
   for (int j = threadIdx.x; j < Lk; j += TAU_THREADS) {
     const float u = zrow[j];
     if (u > m - 1.f) {
       const int k = atomicAdd(&s_n, 1);
-      if (k < cap) cand[k] = u;
+      if (k < cap) {
+        cand[k] = u;
+        cidx[k] = j;
+      }
     }
   }
   __syncthreads();
@@ -527,10 +537,21 @@ __global__ void __launch_bounds__(TAU_THREADS)
   float tau;
   if (n <= cap) {
     tau = block_solve_tau(cand, n, m, P.norm == NATTN_ENTMAX15, red);
+    // pages of the support: the support lies among the candidates
+    for (int k = threadIdx.x; k < n; k += TAU_THREADS)
+      if (cand[k] > tau) {
+        const int pg = cidx[k] / P.page_size;
+        atomicOr(&smask[pg >> 5], 1u << (pg & 31));
+      }
   } else {
     // every masked score is -inf and never enters {u > t}
     tau = block_solve_tau(zrow, Lk, m, P.norm == NATTN_ENTMAX15, red);
+    // too many candidates to track: every page of the row is visited
+    for (int pg = threadIdx.x; pg < npages; pg += TAU_THREADS)
+      atomicOr(&smask[pg >> 5], 1u << (pg & 31));
   }
+  __syncthreads();
+  for (int w = threadIdx.x; w < A.pm_words; w += TAU_THREADS) prow[w] = smask[w];
   if (threadIdx.x == 0) tau_out[row] = tau;
 }
 

@@ -104,7 +104,8 @@ struct Plan {
   size_t off_supc = 0, off_supl = 0;
   int sup_cap = 0;
   bool tc_apply = false;  // sparse phase 2 on the tensor cores (bf16 P)
-  size_t off_opart = 0, off_ml = 0, off_scores = 0;
+  size_t off_opart = 0, off_ml = 0, off_scores = 0, off_pmask = 0;
+  int pm_words = 0;
   size_t total = 0;
   int row_grid = 0, row_cap = 0;
   bool row_slots = false;
@@ -180,6 +181,9 @@ Plan make_plan(const nattn_args* a) {
         off = up256(off + rows * (size_t)a->Tk * 4);
         pl.off_tau = off;
         off = up256(off + rows * 4);
+        pl.pm_words = (maxp + 31) / 32;
+        pl.off_pmask = off;
+        off = up256(off + rows * (size_t)pl.pm_words * 4);
       }
       pl.total = off;
       return pl;
@@ -392,6 +396,8 @@ int launch_decode(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t
   A.ml = reinterpret_cast<float*>(ws + pl.off_ml);
   A.scores = pl.sparse ? reinterpret_cast<float*>(ws + pl.off_scores) : nullptr;
   A.tau = pl.sparse ? reinterpret_cast<float*>(ws + pl.off_tau) : nullptr;
+  A.pmask = pl.sparse ? reinterpret_cast<unsigned*>(ws + pl.off_pmask) : nullptr;
+  A.pm_words = pl.sparse ? pl.pm_words : 0;
   const unsigned rows = (unsigned)((size_t)a->B * a->Hq * a->Tq);
   if (!pl.sparse) {
     A.zscale = a->scale * 1.4426950408889634f;
@@ -405,8 +411,8 @@ int launch_decode(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t
   A.zscale = a->scale * A.uscale;
   int rc = launch_decode_mode<D, PS, DEC_SCORES>(a, A, mk, mv, st);
   if (rc) return rc;
-  const int cap = 16384;
-  const int tbytes = (64 + cap) * 4;
+  const int cap = 12288;  // candidates kept in shared memory (value + key index)
+  const int tbytes = (64 + 2 * cap + pl.pm_words) * 4;
   if (allow_smem(decode_tau_kernel, tbytes) != cudaSuccess) return NATTN_ECUDA;
   decode_tau_kernel<<<rows, TAU_THREADS, tbytes, st>>>(A, const_cast<float*>(A.tau), cap);
   if (check_launch()) return NATTN_ECUDA;
