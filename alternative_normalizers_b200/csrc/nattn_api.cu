@@ -411,7 +411,7 @@ int launch_decode(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t
   A.zscale = a->scale * A.uscale;
   int rc = launch_decode_mode<D, PS, DEC_SCORES>(a, A, mk, mv, st);
   if (rc) return rc;
-  const int cap = 12288;  // candidates kept in shared memory (value + key index)
+  const int cap = 4096;  // candidates kept in shared memory (value + key index)
   const int tbytes = (64 + 2 * cap + pl.pm_words) * 4;
   if (allow_smem(decode_tau_kernel, tbytes) != cudaSuccess) return NATTN_ECUDA;
   decode_tau_kernel<<<rows, TAU_THREADS, tbytes, st>>>(A, const_cast<float*>(A.tau), cap);

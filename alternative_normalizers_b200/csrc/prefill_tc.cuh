@@ -585,7 +585,21 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
             int2* ptr = mybuf + nbuf;
             float sadd = 0.f;
             int na = 0;
-            while (msk && na < room) {
+            // two candidates per trip, so that two stash loads are in flight
+            while (msk && na + 1 < room) {
+              const int k0 = __ffs(msk) - 1;
+              msk &= msk - 1;
+              const int k1 = msk ? __ffs(msk) - 1 : -1;
+              msk &= msk - 1;  // no-op when msk is already 0
+              const float v0 = stash[k0];
+              const float v1 = (k1 >= 0) ? stash[k1] : 0.f;
+              *ptr = make_int2(kj + k0, __float_as_int(v0));
+              if (k1 >= 0) ptr[1] = make_int2(kj + k1, __float_as_int(v1));
+              ptr += (k1 >= 0) ? 2 : 1;
+              sadd += v0 + v1;
+              na += (k1 >= 0) ? 2 : 1;
+            }
+            if (msk && na < room) {  // room for one more
               const int k = __ffs(msk) - 1;
               msk &= msk - 1;
               const float v = stash[k];
