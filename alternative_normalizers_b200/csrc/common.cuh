@@ -68,17 +68,19 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
   return y;
 }
-// Maximum of 32 consecutive values held as raw bits (two three-input chains
-// and a final merge: 16 instructions instead of 31 two-input ones).
+// Maximum of 32 consecutive values held as raw bits: four independent
+// three-input chains of eight values each, then one merge (16 instructions,
+// a dependency depth of five).
 __device__ __forceinline__ float max32_bits(const uint32_t* v) {
-  float a = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
-  float b = fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5]));
+  float c[4];
 #pragma unroll
-  for (int k = 6; k < 30; k += 4) {
-    a = fmax3(a, __uint_as_float(v[k]), __uint_as_float(v[k + 1]));
-    b = fmax3(b, __uint_as_float(v[k + 2]), __uint_as_float(v[k + 3]));
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t* w = v + 8 * q;
+    const float a = fmax3(__uint_as_float(w[0]), __uint_as_float(w[1]), __uint_as_float(w[2]));
+    const float b = fmax3(a, __uint_as_float(w[3]), __uint_as_float(w[4]));
+    c[q] = fmax3(b, __uint_as_float(w[5]), fmaxf(__uint_as_float(w[6]), __uint_as_float(w[7])));
   }
-  return fmax3(a, b, fmaxf(__uint_as_float(v[30]), __uint_as_float(v[31])));
+  return fmaxf(fmaxf(c[0], c[1]), fmaxf(c[2], c[3]));
 }
 
 // ---------------------------------------------------------------------------

@@ -530,10 +530,14 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
         tmem_st_wait();
       } else {  // TC_TAU
         const float vs = fast ? zs : 1.f;  // stored value -> threshold units
+        // chunk maxima first: independent of the bound logic below
+        float cmaxs[LDC / 32];
+#pragma unroll
+        for (int c = 0; c < LDC / 32; ++c) cmaxs[c] = max32_bits(&r[c * 32]) * vs;
 #pragma unroll
         for (int c = 0; c < LDC / 32; ++c) {
           const uint32_t* rc = &r[c * 32];
-          const float cmax = max32_bits(rc) * vs;
+          const float cmax = cmaxs[c];
           m_run = fmaxf(m_run, cmax);
           lb = fmaxf(lb, m_run - 1.f);  // tau >= max - 1
           // The buffer B holds every stored key that can still be in the
@@ -564,12 +568,18 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
           float thr = to_thr(lb);
           // candidate mask: bit k set when value k is above thr, taken from
           // the sign of thr - v (-inf values give +inf: never candidates)
+          // (four independent eight-bit chains, merged at the end)
           auto cand_mask = [&](float t) {
-            unsigned mk = 0;
+            unsigned part[4];
 #pragma unroll
-            for (int k = 31; k >= 0; --k)
-              mk = __funnelshift_l(__float_as_uint(t - __uint_as_float(rc[k])), mk, 1);
-            return mk;
+            for (int q = 0; q < 4; ++q) {
+              unsigned mk = 0;
+#pragma unroll
+              for (int k = 8 * q + 7; k >= 8 * q; --k)
+                mk = __funnelshift_l(__float_as_uint(t - __uint_as_float(rc[k])), mk, 1);
+              part[q] = mk;
+            }
+            return part[0] | (part[1] << 8) | (part[2] << 16) | (part[3] << 24);
           };
           unsigned msk = want ? cand_mask(thr) : 0u;
           // the chunk goes to a per-thread stash so that appends run once per
