@@ -66,10 +66,12 @@ struct TcArgs {
 };
 
 // NH = 2 splits every S row between two warps (columns [0, BN/2) and
-// [BN/2, BN)); each half keeps its own running maximum, denominator and O
-// accumulator in TMEM, and the halves are merged once in the epilogue.  Two
-// normalizer warps per SM sub-partition hide each other's latency and each
-// thread holds half a row in registers.
+// [BN/2, BN)).  In the online mode each half keeps its own running maximum,
+// denominator and O accumulator in TMEM; in the threshold mode each half
+// keeps its own candidate buffer and publishes its running bound for the
+// other.  The halves are merged once in the epilogue.  Two normalizer warps
+// per SM sub-partition hide each other's latency and each thread holds half a
+// row in registers.
 template <int D, int DV, int BN, int KST, int VST, int MODE, int NH = 1>
 struct TcLayout {
   static_assert(NH == 1 || MODE != TC_APPLY, "row split is for the online and tau modes");
@@ -101,7 +103,7 @@ struct TcLayout {
   static constexpr int OFF_XCH = OFF_Q;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
-  // TMEM columns: S double buffer, then O
+  // TMEM columns: the S ring (NSB buffers of BN columns), then O
   static constexpr int TM_S = 0;  // S buffer s at column s * BN
   static constexpr int TM_O = 2 * BN;
   static constexpr int TM_COLS_USED = (MODE == TC_TAU) ? NSB * BN : 2 * BN + NH * DV;
