@@ -15,6 +15,7 @@ from .binding import (  # noqa: F401
     nattn_fwd,
     nattn_fwd_ex,
     nattn_get_device_status,
+    nattn_selftest_wait_timeout,
     nattn_strerror,
     nattn_version,
     nattn_workspace_size,

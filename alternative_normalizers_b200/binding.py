@@ -81,6 +81,8 @@ def lib():
         L.nattn_version.restype = ctypes.c_int
         L.nattn_decode_noalloc.argtypes = [P]
         L.nattn_decode_noalloc.restype = ctypes.c_int
+        L.nattn_selftest_wait_timeout.argtypes = [ctypes.c_void_p]
+        L.nattn_selftest_wait_timeout.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -116,6 +118,12 @@ def nattn_strerror(code):
 
 def nattn_version():
     return lib().nattn_version()
+
+
+def nattn_selftest_wait_timeout(stream=None):
+    """Launch the bounded-wait self-test: one wait that nothing completes,
+    which gives up after about two seconds and records NATTN_ETIMEOUT."""
+    return lib().nattn_selftest_wait_timeout(stream)
 
 
 def nattn_decode_noalloc(args: NattnArgs):

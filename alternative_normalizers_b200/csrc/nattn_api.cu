@@ -528,6 +528,24 @@ int decode_noalloc(const nattn_args* a) {
 
 }  // namespace
 
+namespace nattn {
+// One bounded wait on an mbarrier phase that nothing completes: the wait
+// gives up after its budget and records NATTN_ETIMEOUT (see
+// nattn_selftest_wait_timeout in the header).
+__global__ void selftest_wait_kernel() {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_addr(&bar), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) mbar_wait(smem_addr(&bar), 0, &abort_flag);
+  __syncwarp();
+}
+}  // namespace nattn
+
 extern "C" {
 
 __attribute__((visibility("default"))) int nattn_fwd_ex(const nattn_args* a) { return run(a); }
@@ -606,6 +624,11 @@ __attribute__((visibility("default"))) const char* nattn_strerror(int code) {
     case NATTN_EALIGN: return "pointer not 16-byte aligned";
     default: return "unknown error";
   }
+}
+
+__attribute__((visibility("default"))) int nattn_selftest_wait_timeout(void* stream) {
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return check_launch();
 }
 
 __attribute__((visibility("default"))) int nattn_version(void) { return kVersion; }

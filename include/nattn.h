@@ -201,6 +201,24 @@ const char* nattn_strerror(int code);
 #define NATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
 int nattn_decode_noalloc(const nattn_args* a);
 
+/*
+ * Self-test of the bounded-wait failure path (no paper counterpart; a test
+ * hook of this library).
+ *
+ * Every wait of the kernels above on an mbarrier phase is bounded: after
+ * about two seconds it records NATTN_ETIMEOUT in the device status word, lets
+ * the other roles of its CTA stop, and returns, so the CUDA context stays
+ * usable.  This entry point launches one CTA whose thread waits, with that
+ * same bounded wait, on an mbarrier that nothing ever completes, and so
+ * exercises the path without faulting, trapping or hanging the GPU.
+ *
+ * Asynchronous on `stream` (NULL: the default stream); the kernel runs for
+ * about two seconds.  Returns NATTN_OK if the launch succeeded, else
+ * NATTN_ECUDA.  Afterwards nattn_get_device_status(stream) returns
+ * NATTN_ETIMEOUT (and clears it).
+ */
+int nattn_selftest_wait_timeout(void* stream);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 int nattn_version(void);
 
