@@ -94,6 +94,8 @@ TC_CASES = [
     (1, 2, 1, 600, 600, 128, True, 256, 0.0),    # sliding window
     (1, 2, 1, 300, 300, 128, True, 1000, 1.0),   # window >= T, heavy cap
     (1, 2, 1, 130, 130, 128, False, 50, 0.0),    # two-sided window
+    (2, 4, 2, 1, 500, 128, True, 0, 0.0),        # one query row over 500 keys
+    (1, 4, 4, 17, 1, 64, False, 0, 0.0),         # a single key
 ]
 
 
