@@ -28,7 +28,7 @@ class NattnArgs(ctypes.Structure):
     _fields_ = [
         ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
         ("out", ctypes.c_void_p), ("row_stat", ctypes.c_void_p),
-        ("weights", ctypes.c_void_p),
+        ("weights", ctypes.c_void_p), ("row_nnz", ctypes.c_void_p),
         ("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
         ("Tq", ctypes.c_int), ("Tk", ctypes.c_int), ("d", ctypes.c_int),
         ("dv", ctypes.c_int),
@@ -149,13 +149,16 @@ def _norm_id(normalizer):
 def build_args(q, k, v, out, row_stat=None, weights=None, *, normalizer,
                causal=False, window=0, softcap=0.0, scale=None,
                block_table=None, seqlens=None, page_size=0, max_seqlen=None,
-               stream=None):
-    """Fill an ``NattnArgs`` from torch tensors (no device work)."""
+               stream=None, row_nnz=None):
+    """Fill an ``NattnArgs`` from torch tensors (no device work).
+    ``row_nnz`` (int32 [B, Hq, Tq] or None) receives the number of keys with
+    a nonzero weight in each row."""
     import torch
     B, Hq, Tq, d = q.shape
     a = NattnArgs()
     a.q, a.k, a.v, a.out = _ptr(q), _ptr(k), _ptr(v), _ptr(out)
     a.row_stat, a.weights = _ptr(row_stat), _ptr(weights)
+    a.row_nnz = _ptr(row_nnz)
     a.B, a.Hq, a.Tq, a.d = B, Hq, Tq, d
     a.Hkv = k.shape[1]
     a.dv = v.shape[3]
@@ -191,10 +194,10 @@ def _run(a, workspace_holder):
 
 def attention(q, k, v, normalizer="softmax", causal=False, window=0,
               softcap=0.0, scale=None, want_weights=False, out=None,
-              row_stat=None):
+              row_stat=None, row_nnz=None):
     """Dense attention forward.  q [B,Hq,Tq,d], k [B,Hkv,Tk,d], v
     [B,Hkv,Tk,dv] (bf16, CUDA, contiguous).  Returns (out, row_stat,
-    weights|None)."""
+    weights|None); fills ``row_nnz`` (int32 [B,Hq,Tq]) when given."""
     import torch
     B, Hq, Tq, _ = q.shape
     Tk, dv = k.shape[2], v.shape[3]
@@ -205,7 +208,8 @@ def attention(q, k, v, normalizer="softmax", causal=False, window=0,
     weights = torch.empty(B, Hq, Tq, Tk, dtype=torch.float32,
                           device=q.device) if want_weights else None
     a = build_args(q, k, v, out, row_stat, weights, normalizer=normalizer,
-                   causal=causal, window=window, softcap=softcap, scale=scale)
+                   causal=causal, window=window, softcap=softcap, scale=scale,
+                   row_nnz=row_nnz)
     keep = []
     _run(a, keep)
     return out, row_stat, weights
@@ -213,10 +217,10 @@ def attention(q, k, v, normalizer="softmax", causal=False, window=0,
 
 def paged_attention(q, k_pool, v_pool, block_table, seqlens, max_seqlen,
                     normalizer="softmax", causal=True, window=0, softcap=0.0,
-                    scale=None, out=None, row_stat=None):
+                    scale=None, out=None, row_stat=None, row_nnz=None):
     """Attention of q [B,Hq,Tq,d] over a paged cache: k_pool/v_pool
     [num_pages, Hkv, page, d], block_table int32 [B, max_pages], seqlens
-    int32 [B] (each <= max_seqlen)."""
+    int32 [B] (each <= max_seqlen).  Fills ``row_nnz`` when given."""
     import torch
     B, Hq, Tq, _ = q.shape
     dv = v_pool.shape[3]
@@ -228,7 +232,7 @@ def paged_attention(q, k_pool, v_pool, block_table, seqlens, max_seqlen,
                    normalizer=normalizer, causal=causal, window=window,
                    softcap=softcap, scale=scale, block_table=block_table,
                    seqlens=seqlens, page_size=k_pool.shape[2],
-                   max_seqlen=max_seqlen)
+                   max_seqlen=max_seqlen, row_nnz=row_nnz)
     keep = []
     _run(a, keep)
     return out, row_stat

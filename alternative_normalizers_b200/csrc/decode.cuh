@@ -468,6 +468,10 @@ __global__ void decode_combine_kernel(DecodeArgs A, int mode) {
     }
     if (threadIdx.x == 0 && P.row_stat)
       P.row_stat[row] = (l > 0.f) ? (msafe + log2f(l)) * 0.6931471805599453f : -INFINITY;
+    if (threadIdx.x == 0 && P.row_nnz) {
+      const RowRange rr = row_range(P, i, valid ? Lk : 0);
+      P.row_nnz[row] = rr.hi >= rr.lo ? rr.hi - rr.lo + 1 : 0;
+    }
   } else {
     for (int c = threadIdx.x; c < P.dv; c += blockDim.x) {
       float o = 0.f;
@@ -493,6 +497,7 @@ __global__ void __launch_bounds__(TAU_THREADS)
   int* cidx = reinterpret_cast<int*>(cand + cap);             // [cap] key indices
   unsigned* smask = reinterpret_cast<unsigned*>(cidx + cap);  // [pm_words]
   __shared__ int s_n;
+  __shared__ int s_sup;  // support size
   const Problem& P = A.P;
   const int row = blockIdx.x;
   const int i = row % P.Tq;
@@ -505,6 +510,7 @@ __global__ void __launch_bounds__(TAU_THREADS)
   unsigned* prow = A.pmask + (size_t)row * A.pm_words;
   if (!valid) {
     if (threadIdx.x == 0) tau_out[row] = INFINITY;
+    if (threadIdx.x == 0 && P.row_nnz) P.row_nnz[row] = 0;
     for (int w = threadIdx.x; w < A.pm_words; w += TAU_THREADS) prow[w] = 0u;
     return;
   }
@@ -515,10 +521,14 @@ __global__ void __launch_bounds__(TAU_THREADS)
   for (int s = 0; s < nact; ++s) m = fmaxf(m, A.ml[(pbase + (size_t)s * A.R) * 2]);
   if (m == -INFINITY) {  // no visible key
     if (threadIdx.x == 0) tau_out[row] = INFINITY;
+    if (threadIdx.x == 0 && P.row_nnz) P.row_nnz[row] = 0;
     for (int w = threadIdx.x; w < A.pm_words; w += TAU_THREADS) prow[w] = 0u;
     return;
   }
-  if (threadIdx.x == 0) s_n = 0;
+  if (threadIdx.x == 0) {
+    s_n = 0;
+    s_sup = 0;
+  }
   for (int w = threadIdx.x; w < A.pm_words; w += TAU_THREADS) smask[w] = 0u;
   __syncthreads();
   const float* zrow = A.scores + (size_t)row * P.Tk;
@@ -542,6 +552,7 @@ __global__ void __launch_bounds__(TAU_THREADS)
       if (cand[k] > tau) {
         const int pg = cidx[k] / P.page_size;
         atomicOr(&smask[pg >> 5], 1u << (pg & 31));
+        atomicAdd(&s_sup, 1);
       }
   } else {
     // every masked score is -inf and never enters {u > t}
@@ -549,8 +560,11 @@ __global__ void __launch_bounds__(TAU_THREADS)
     // too many candidates to track: every page of the row is visited
     for (int pg = threadIdx.x; pg < npages; pg += TAU_THREADS)
       atomicOr(&smask[pg >> 5], 1u << (pg & 31));
+    for (int j = threadIdx.x; j < Lk; j += TAU_THREADS)
+      if (zrow[j] > tau) atomicAdd(&s_sup, 1);
   }
   __syncthreads();
+  if (threadIdx.x == 0 && P.row_nnz) P.row_nnz[row] = s_sup;
   for (int w = threadIdx.x; w < A.pm_words; w += TAU_THREADS) prow[w] = smask[w];
   if (threadIdx.x == 0) tau_out[row] = tau;
 }

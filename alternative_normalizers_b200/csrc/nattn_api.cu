@@ -240,6 +240,7 @@ Problem to_problem(const nattn_args* a) {
   P.out = static_cast<bf16*>(a->out);
   P.row_stat = a->row_stat;
   P.weights = a->weights;
+  P.row_nnz = a->row_nnz;
   P.B = a->B;
   P.Hq = a->Hq;
   P.Hkv = a->Hkv;

@@ -205,6 +205,7 @@ __device__ __forceinline__ void prefill_pair_normalizer(
     }
   }
   if (row_ok && P.row_stat) P.row_stat[flat] = stat;
+  if (row_ok && P.row_nnz) P.row_nnz[flat] = rr.hi >= rr.lo ? rr.hi - rr.lo + 1 : 0;
 }
 
 template <int D, int KST, int VST>

@@ -706,6 +706,8 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
         }
         A.tau[flat] = t;
         A.sup_count[flat] = nsup;
+        // rows sent to the row-wise pass get their count there
+        if (!ovf_r && P.row_nnz) P.row_nnz[flat] = nsup;
       }
     } else {
       const bool have_o =
@@ -770,6 +772,10 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
         }
       }
       if (row_ok && P.row_stat && half == 0) P.row_stat[flat] = stat;
+      if constexpr (MODE == TC_ONLINE) {
+        if (row_ok && P.row_nnz && half == 0)
+          P.row_nnz[flat] = rr.hi >= rr.lo ? rr.hi - rr.lo + 1 : 0;
+      }
     }
   }
 

@@ -14,6 +14,7 @@ struct Problem {
   bf16* out;
   float* row_stat;
   float* weights;
+  int32_t* row_nnz;  // keys with a nonzero weight per row, or null
   int B, Hq, Hkv, Tq, Tk, d, dv;
   float scale;
   int norm;

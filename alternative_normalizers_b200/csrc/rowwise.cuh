@@ -233,6 +233,7 @@ __global__ void __launch_bounds__(ROW_THREADS)
 
     // normalizer: overwrite scores with weights
     float stat;
+    int nnz = n;  // softmax / softmax1: every visible key
     if (P.norm == NATTN_SOFTMAX || P.norm == NATTN_SOFTMAX1) {
       float mx = -INFINITY;
       for (int jj = tid; jj < n; jj += ROW_THREADS) mx = fmaxf(mx, sc[jj]);
@@ -277,10 +278,13 @@ __global__ void __launch_bounds__(ROW_THREADS)
                                : block_solve_tau(sc, n, mx, ent, red);
       }
       __syncthreads();
+      float cnt = 0.f;
       for (int jj = tid; jj < n; jj += ROW_THREADS) {
         const float t = fmaxf(sc[jj] - tau, 0.f);
         sc[jj] = ent ? t * t : t;
+        cnt += (t > 0.f) ? 1.f : 0.f;
       }
+      nnz = (int)block_sum(cnt, red);
       stat = tau;
     }
     __syncthreads();
@@ -357,6 +361,7 @@ __global__ void __launch_bounds__(ROW_THREADS)
       }
     }
     if (tid == 0 && P.row_stat) P.row_stat[flat] = stat;
+    if (tid == 0 && P.row_nnz) P.row_nnz[flat] = nnz;
     __syncthreads();
   }
 }

@@ -107,6 +107,10 @@ enum {
  *            tau in units of z/2 (+inf for such a row).
  *   weights  float32 [B, Hq, Tq, Tk] dense attention weights or NULL (dense
  *            mode only, at most 2^26 entries; masked entries are exactly 0).
+ *   row_nnz  int32 [B, Hq, Tq] or NULL: keys with a nonzero weight in each
+ *            row.  sparsemax / entmax15: the support size (every other
+ *            visible key has a weight of exactly 0); softmax / softmax1: the
+ *            number of visible keys.  0 for a row with no visible key.
  *
  * window == 0 disables the sliding window; with causal it keeps keys with
  * 0 <= pos - j < window ("attention interface" wiki, section "common
@@ -120,6 +124,7 @@ typedef struct nattn_args {
   void* out;
   float* row_stat;
   float* weights;
+  int32_t* row_nnz;
   int B, Hq, Hkv, Tq, Tk, d, dv;
   float scale;
   int normalizer;
