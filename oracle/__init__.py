@@ -26,7 +26,7 @@ Every function cites the passage of the source pages it restates:
 * "HF Attention Normalizers", section "Packed Variable-Length Attention"
   (bottom-right causal alignment when query and key lengths differ).
 
-Readings where the pages are silent (all listed in the design doc):
+Readings where the pages are silent:
 sparsemax is the Euclidean projection onto the probability simplex;
 1.5-entmax is ``p_i = relu(z_i/2 - tau)^2`` with ``sum p = 1`` and its
 threshold is reported in units of ``z/2``; scores are scaled, then soft-capped,
