@@ -129,7 +129,8 @@ int validate(const nattn_args* a) {
   if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out))
     return NATTN_EALIGN;
   if ((a->row_stat && (reinterpret_cast<uintptr_t>(a->row_stat) & 3)) ||
-      (a->weights && (reinterpret_cast<uintptr_t>(a->weights) & 3)))
+      (a->weights && (reinterpret_cast<uintptr_t>(a->weights) & 3)) ||
+      (a->row_nnz && (reinterpret_cast<uintptr_t>(a->row_nnz) & 3)))
     return NATTN_EALIGN;
   const long long rows = (long long)a->B * a->Hq * a->Tq;
   if (rows >= (1ll << 31) || rows * (long long)(a->d > a->dv ? a->d : a->dv) >= (1ll << 40))

@@ -62,8 +62,8 @@ enum {
   NATTN_EINVAL = -1,        /* bad argument: NULL pointer, negative size,
                                Hq % Hkv != 0, non-finite scale, ...        */
   NATTN_EUNSUPPORTED = -2,  /* well-formed but outside what the kernels do:
-                               head dim not in {32, 64, 128, 256}, paged mode
-                               with dense weights, ...                       */
+                               d or dv not a multiple of 8 in [8, 256],
+                               paged mode with dense weights, ...            */
   NATTN_ETOOLARGE = -3,     /* dense weights asked for more than 2^26 entries,
                                or a size beyond the int32 index range       */
   NATTN_EWORKSPACE = -4,    /* workspace NULL or smaller than
@@ -73,7 +73,9 @@ enum {
   NATTN_EBOUNDS = -7,       /* device: a block-table entry or a sequence
                                length was out of range; the offending work
                                item wrote zeros and was skipped             */
-  NATTN_EALIGN = -8         /* a pointer is not 16-byte aligned             */
+  NATTN_EALIGN = -8         /* q, k, v, out or workspace not 16-byte
+                               aligned, or row_stat, weights or row_nnz not
+                               4-byte aligned                                */
 };
 
 /*

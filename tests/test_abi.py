@@ -59,6 +59,8 @@ def _args(L, **kw):
     (dict(scale=float("nan")), -1), (dict(scale=float("inf")), -1),
     (dict(softcap=-1.0), -1), (dict(window=-2), -1), (dict(normalizer=4), -1),
     (dict(causal=2), -1), (dict(B=-1), -1), (dict(q=4100), -8),
+    (dict(row_stat=4098), -8), (dict(row_nnz=4098), -8), (dict(d=12), -2),
+    (dict(dv=264), -2),
 ])
 def test_host_validation(L, kw, code):
     a = _args(L, **kw)
