@@ -80,6 +80,34 @@ bool make_map_2d(CUtensorMap* m, const void* base, int inner, long long rows, in
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Driver entry points looked up by name through the runtime (no -lcuda).
+template <class F>
+F driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion(name, &p, 12000, cudaEnableDefault, &q) ==
+          cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<F>(p);
+  return nullptr;
+}
+
+typedef CUresult (*AddrRangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
+typedef CUresult (*CtxCurrentFn)(CUcontext*);
+typedef CUresult (*CtxIdFn)(CUcontext, unsigned long long*);
+
+// Bytes from `p` to the end of the device allocation that contains it, or 0
+// when `p` is not inside a device allocation of this process.
+size_t bytes_to_alloc_end(const void* p) {
+  static AddrRangeFn fn = driver_fn<AddrRangeFn>("cuMemGetAddressRange");
+  if (!fn) return 0;
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (fn(&base, &size, reinterpret_cast<CUdeviceptr>(p)) != CUDA_SUCCESS) return 0;
+  const CUdeviceptr at = reinterpret_cast<CUdeviceptr>(p);
+  return (at >= base && at < base + size) ? (size_t)(base + size - at) : 0;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -103,7 +131,6 @@ struct Plan {
   size_t off_tau = 0, off_ovfc = 0, off_ovfr = 0, off_slots = 0;
   size_t off_supc = 0, off_supl = 0;
   int sup_cap = 0;
-  bool tc_apply = false;  // sparse phase 2 on the tensor cores (bf16 P)
   size_t off_opart = 0, off_ml = 0, off_scores = 0, off_pmask = 0;
   int pm_words = 0;
   size_t total = 0;
@@ -149,11 +176,10 @@ int validate(const nattn_args* a) {
   return NATTN_OK;
 }
 
-int decode_pps() {
-  const char* e = getenv("NATTN_DECODE_PPS");
-  int v = e ? atoi(e) : 0;
-  return (v >= 1 && v <= 256) ? v : 32;
-}
+// Pages per decode split: 32 pages (2048 keys at 64-token pages) keeps every
+// CTA's loads several pages deep while the (sequence, kv head, split) grid of
+// the decode workload still fills two CTAs per SM many times over.
+constexpr int kDecodePagesPerSplit = 32;
 
 Plan make_plan(const nattn_args* a) {
   Plan pl;
@@ -168,7 +194,7 @@ Plan make_plan(const nattn_args* a) {
       pl.path = PATH_DECODE;
       pl.R = group * a->Tq;
       const int maxp = (a->Tk + a->page_size - 1) / a->page_size;
-      pl.pps = decode_pps();
+      pl.pps = kDecodePagesPerSplit;
       if (pl.pps > maxp) pl.pps = maxp;
       pl.nsplit = (maxp + pl.pps - 1) / pl.pps;
       const size_t parts = (size_t)a->B * a->Hkv * pl.nsplit * pl.R;
@@ -204,10 +230,6 @@ Plan make_plan(const nattn_args* a) {
       off = up256(off + rows * 4);
       pl.off_supl = off;
       off = up256(off + rows * (size_t)pl.sup_cap * 8);
-      {
-        const char* e = getenv("NATTN_SPARSE_APPLY");
-        pl.tc_apply = e && strcmp(e, "tc") == 0;
-      }
       pl.row_grid = 2 * 148;
       pl.row_cap = a->Tk < kRowSmemCap ? (a->Tk < 256 ? 256 : a->Tk) : kRowSmemCap;
       if (a->Tk > kRowSmemCap) {
@@ -343,13 +365,8 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
     k<<<grid, LY::THREADS, LY::ALLOC, st>>>(mq, mk, mv, A);
     if (check_launch() != NATTN_OK) return NATTN_ECUDA;
   }
-  if (pl.tc_apply) {
-    using LY = TcLayout<D, D, BN, KST, VST, TC_APPLY>;
-    auto k = prefill_tc_kernel<D, D, BN, KST, VST, TC_APPLY>;
-    if (allow_smem(k, LY::ALLOC) != cudaSuccess) return NATTN_ECUDA;
-    k<<<grid, LY::THREADS, LY::ALLOC, st>>>(mq, mk, mv, A);
-    if (check_launch() != NATTN_OK) return NATTN_ECUDA;
-  } else {
+  {
+    // phase 2: fp32 gather over each row's support list
     const size_t rows = (size_t)a->B * a->Hq * a->Tq;
     const unsigned g2 = (unsigned)((rows + GATHER_WARPS - 1) / GATHER_WARPS);
     sparse_gather_kernel<D><<<g2, GATHER_WARPS * 32, 0, st>>>(P, A.sup_count, A.sup_list,
@@ -368,7 +385,8 @@ int launch_decode_mode(const nattn_args* a, const DecodeArgs& A, const CUtensorM
   // about 100 KB of stages: two CTAs per SM for K+V pages, three for K or V
   constexpr int NS = (L1::STAGE * 4 <= 100 * 1024) ? 4 : (L1::STAGE * 3 <= 100 * 1024 ? 3 : 2);
   using L = DecodeSmem<D, D, PS, NS, MODE>;
-  const int bytes = L::BYTES_NOLIST + 2 * A.pps * 4 + 1024;
+  // only the sparse apply pass keeps a page list (two ints per page)
+  const int bytes = L::BYTES_NOLIST + (MODE == DEC_APPLY ? 2 * A.pps * 4 : 0) + 1024;
   dim3 grid(A.nsplit, a->Hkv, a->B);
   if (A.R <= 8) {
     auto k = decode_split_kernel<D, D, PS, NS, 1, MODE>;
@@ -470,19 +488,37 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[NATTN_NOALLOC_S
 constexpr int kNoAllocDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_addr[kNoAllocDevices] = {};
+unsigned long long g_noalloc_ctx[kNoAllocDevices] = {};  // context id of the lookup
 
-// Device address of the scratch array on the current device (first call per
-// device does the lookup with that device current).
+// Device address of the scratch array on the current device.  The first call
+// per device does the lookup with that device current; the address is kept
+// with the id of the context it belongs to and looked up again whenever the
+// device's current context is a different one (after cudaDeviceReset, for
+// instance, the module is loaded anew and the array may move).
 int noalloc_scratch(void** out) {
+  static CtxCurrentFn ctx_current = driver_fn<CtxCurrentFn>("cuCtxGetCurrent");
+  static CtxIdFn ctx_id = driver_fn<CtxIdFn>("cuCtxGetId");
+  if (!ctx_current || !ctx_id) return NATTN_ECUDA;
+  auto current_id = [&](unsigned long long* id) {
+    CUcontext ctx = nullptr;
+    return ctx_current(&ctx) == CUDA_SUCCESS && ctx != nullptr &&
+           ctx_id(ctx, id) == CUDA_SUCCESS;
+  };
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocDevices)
     return NATTN_ECUDA;
+  unsigned long long id = 0;
+  // false before the runtime has bound its context to this thread; the
+  // symbol lookup below does that
+  const bool have_id = current_id(&id);
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_addr[dev] == nullptr) {
+  if (!have_id || g_noalloc_addr[dev] == nullptr || g_noalloc_ctx[dev] != id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return NATTN_ECUDA;
+    if (!have_id && !current_id(&id)) return NATTN_ECUDA;
     g_noalloc_addr[dev] = p;
+    g_noalloc_ctx[dev] = id;
   }
   *out = g_noalloc_addr[dev];
   return NATTN_OK;
@@ -587,10 +623,22 @@ __attribute__((visibility("default"))) int nattn_fwd(const void* q, const void* 
   if (block_table) {
     a.page_size = 64;
     a.block_table_stride = (Tk + 63) / 64;
-    a.num_pages = 0x7fffffff / (Hkv > 0 ? Hkv * 64 : 64);
+    a.num_pages = 1;  // placeholder for the host checks below
   }
   int rc = validate(&a);
   if (rc != NATTN_OK) return rc;
+  if (block_table && B > 0 && Hq > 0 && Tq > 0) {
+    // The pool holds as many whole pages as the device allocations that
+    // contain k and v reach past their start: page ids at or past that bound
+    // are caught on the device (NATTN_EBOUNDS), so a bad table never reads
+    // memory this process does not own.
+    const size_t kb = bytes_to_alloc_end(k), vb = bytes_to_alloc_end(v);
+    const size_t kpage = (size_t)Hkv * 64 * d * 2, vpage = (size_t)Hkv * 64 * dv * 2;
+    size_t np = kb / kpage < vb / vpage ? kb / kpage : vb / vpage;
+    if (np < 1) return NATTN_EINVAL;
+    const size_t cap = (size_t)((1ll << 31) - 1) / ((size_t)Hkv * 64);
+    a.num_pages = (int)(np < cap ? np : cap);
+  }
   const size_t need = nattn_workspace_size(&a);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (need > 0) {

@@ -34,8 +34,8 @@
 //           stream K/V tiles, solve the global normalization threshold and
 //           save one threshold per query row).  Rows whose candidates
 //           overflow the buffer are listed for the row-wise kernel.
-//   APPLY   sparse phase 2: p = relu(z - tau) or relu(z/2 - tau)^2 with tau
-//           fixed, O += P V; no maximum, no division, no rescale.
+// Sparse phase 2 is sparse_gather_kernel below: an fp32 sum over each row's
+// support list.
 #pragma once
 
 #include "common.cuh"
@@ -43,7 +43,7 @@
 
 namespace nattn {
 
-enum TcMode { TC_ONLINE = 0, TC_TAU = 1, TC_APPLY = 2 };
+enum TcMode { TC_ONLINE = 0, TC_TAU = 1 };
 
 constexpr int TC_THREADS = 192;
 constexpr int TC_BM = 128;
@@ -55,9 +55,9 @@ struct TauCap {
 
 struct TcArgs {
   Problem P;
-  float zscale;      // ONLINE: scale * log2(e); TAU/APPLY: scale * uscale
+  float zscale;      // ONLINE: scale * log2(e); TAU: scale * uscale
   float capscale;    // soft-cap: z = capscale * tanh(s * scale / cap)
-  float* tau;        // [B*Hq*Tq]: written by TAU, read by APPLY
+  float* tau;        // [B*Hq*Tq]: written by TAU, read by the gather
   int* ovf_rows;     // TAU: rows whose candidate buffer overflowed
   int* ovf_count;    // TAU: number of such rows (zeroed before the launch)
   int* sup_count;    // TAU: support size of every row (0 for overflowed rows)
@@ -74,7 +74,6 @@ struct TcArgs {
 // row in registers.
 template <int D, int DV, int BN, int KST, int VST, int MODE, int NH = 1>
 struct TcLayout {
-  static_assert(NH == 1 || MODE != TC_APPLY, "row split is for the online and tau modes");
   static constexpr int NWN = 4 * NH;                 // normalizer warps
   static constexpr int THREADS = (NWN + 2) * 32;     // + TMA warp + MMA warp
   static constexpr int QBYTES = D * TC_BM * 2;
@@ -408,7 +407,6 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
     } else {
       m_run = -INFINITY;
     }
-    if constexpr (MODE == TC_APPLY) tau = row_ok ? A.tau[flat] : INFINITY;
     const bool entmax = P.norm == NATTN_ENTMAX15;
     bool alive = true;
 
@@ -511,25 +509,6 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
           tmem_st_wait();
         }
         m_run = m_use;
-      } else if constexpr (MODE == TC_APPLY) {
-        // p = relu(z - tau) or relu(z/2 - tau)^2 as bf16 P
-        const float fa = fast ? zs : 1.f;
-#pragma unroll
-        for (int c = 0; c < LDC / 64; ++c) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int k = 0; k < 64; k += 2) {
-            float x0 = fmaxf(fmaf(__uint_as_float(r[c * 64 + k]), fa, -tau), 0.f);
-            float x1 = fmaxf(fmaf(__uint_as_float(r[c * 64 + k + 1]), fa, -tau), 0.f);
-            if (entmax) {
-              x0 *= x0;
-              x1 *= x1;
-            }
-            pk[k >> 1] = pack_bf16(x0, x1);
-          }
-          tmem_st32(paddr + c * 32, pk);
-        }
-        tmem_st_wait();
       } else {  // TC_TAU
         const float vs = fast ? zs : 1.f;  // stored value -> threshold units
         // chunk maxima first: independent of the bound logic below

@@ -105,6 +105,68 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+class NvmlSampler:
+    """SM clock and clock-event reasons of one GPU, polled through NVML
+    every ``period_s`` on a background thread (read-only queries), so that
+    even a timed region of a few milliseconds holds several samples.  Falls
+    back to the nvidia-smi sampler when NVML is not usable."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, device, period_s=0.002):
+        self.device = device
+        self.period = period_s
+        self.rows = []
+        self.thread = None
+        self.fallback = None
+
+    def start(self):
+        import threading
+        try:
+            import pynvml as N
+            import torch
+            N.nvmlInit()
+            idx = torch.cuda._get_nvml_device_index(self.device)
+            h = N.nvmlDeviceGetHandleByIndex(idx)
+            smax = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
+            bits = [(n, getattr(N, a)) for n, a in self.REASONS]
+        except Exception:
+            self.fallback = ClockSampler(int(getattr(self.device, "index", 0) or 0))
+            self.fallback.start()
+            return
+        self.stop_evt = threading.Event()
+
+        def loop():
+            while not self.stop_evt.is_set():
+                try:
+                    sm = N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)
+                    rs = N.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.rows.append((sm, smax, [n for n, b in bits if rs & b]))
+                except Exception:
+                    pass
+                self.stop_evt.wait(self.period)
+
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        if self.fallback is not None:
+            return self.fallback.stop()
+        if self.thread is None:
+            return None
+        self.stop_evt.set()
+        self.thread.join(timeout=5)
+        if not self.rows:
+            return None
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows),
+                "sm_max_mhz": max(r[1] for r in self.rows),
+                "reasons": sorted({x for r in self.rows for x in r[2]}),
+                "samples": len(self.rows), "source": "nvml"}
+
+
 # --------------------------------------------------------------------------
 # native arm
 # --------------------------------------------------------------------------
@@ -334,7 +396,7 @@ def main_native(args):
     if binding.nattn_get_device_status() != 0:
         raise RuntimeError("device status after warm-up")
 
-    sampler = ClockSampler(local)
+    sampler = NvmlSampler(dev)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -528,8 +590,17 @@ def detail(args, dev, flush):
             else:
                 vals = {n: round(u / (t * 1e-3) / 1e12, 1) for n, t in per.items()}
                 unit = "useful TFLOP/s"
+            peaks = load_peaks()[0]
+            if w.paged:
+                frac = {n: round(v / peaks["hbm_gbs"], 4) for n, v in vals.items()}
+                fkind = "of measured hbm_gbs (dense-equivalent bytes)"
+            else:
+                frac = {n: round(v / peaks["bf16_tflops"], 4)
+                        for n, v in vals.items()}
+                fkind = "of measured bf16_tflops (burst)"
             res[name] = {"unit": unit, "value": vals,
-                         "ms": {n: round(t, 4) for n, t in per.items()}}
+                         "ms": {n: round(t, 4) for n, t in per.items()},
+                         "roofline_frac": frac, "roofline_denominator": fkind}
             sparse = [n for n in per if n in ("sparsemax", "entmax15")]
             if w.paged and sparse:
                 peak = load_peaks()[0]["hbm_gbs"]
@@ -589,6 +660,19 @@ def main_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def spawn_ranks(n):
+    """Run this same command as ``n`` ranks, one per GPU, under
+    torch.distributed.run (rendezvous on 127.0.0.1); returns its exit code."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1",
+           "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
@@ -608,6 +692,11 @@ def main():
     args = p.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is not None and int(env_world) != args.gpus:
+        sys.exit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={env_world}")
+    if env_world is None and args.gpus > 1:
+        sys.exit(spawn_ranks(args.gpus))
     if args.impl == "reference":
         main_reference(args)
     else:

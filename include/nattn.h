@@ -144,11 +144,23 @@ typedef struct nattn_args {
 } nattn_args;
 
 /*
- * Attention forward with the argument list of the backend contract.
+ * Attention forward with the argument list of the backend contract
+ * ("Attention", factory.ai transformers wiki, section "What every backend
+ * must support"; paged arguments as in "HF Attention Normalizers", section
+ * "Differentiable Paged Attention").
+ *
  * Dense mode when block_table == NULL.  In paged mode this short form fixes
- * page_size = 64, block_table_stride = ceil(Tk / 64) and does not bound the
- * page ids from above (use nattn_fwd_ex for other layouts).  Scratch the
- * chosen path needs is allocated and freed stream-ordered on `stream`.
+ * page_size = 64 and block_table_stride = ceil(Tk / 64), and takes the pool
+ * size from the device allocations that hold k and v: the pool has as many
+ * whole pages [Hkv, 64, d] (and [Hkv, 64, dv]) as fit between k (and v) and
+ * the end of the allocation containing it (cuMemGetAddressRange).  A page id
+ * at or past that bound is caught on the device (NATTN_EBOUNDS; that row's
+ * work is skipped), so a bad table never reads memory the process does not
+ * own; with a sub-allocating allocator the bound is the enclosing segment,
+ * not the tensor.  k or v outside any device allocation of this process:
+ * NATTN_EINVAL.  Use nattn_fwd_ex for other page sizes, strides or an exact
+ * page count.  Scratch the chosen path needs is allocated and freed
+ * stream-ordered (cudaMallocAsync / cudaFreeAsync) on `stream`.
  * Returns NATTN_OK or a negative error code.
  */
 int nattn_fwd(const void* q, const void* k, const void* v, void* out,
@@ -191,13 +203,19 @@ const char* nattn_strerror(int code);
  *   - Supported: paged mode, NATTN_SOFTMAX or NATTN_SOFTMAX1, d == dv in
  *     {64, 128, 256}, page_size 32 or 64, (Hq / Hkv) * Tq <= 16.  Anything
  *     else returns NATTN_EUNSUPPORTED.
- *   - The split count is chosen so the partials fit the array; a batch whose
- *     partials do not fit even with one split per sequence
- *     (B * Hkv * (Hq / Hkv) * Tq * (dv + 2) * 4 bytes > the array) returns
- *     NATTN_ETOOLARGE and launches nothing.
+ *   - The split count is chosen so the partials fit the array.  With
+ *     rows = B * Hq * Tq, one split needs
+ *         up256(rows * dv * 4) + up256(rows * 8)
+ *     bytes, where up256 rounds up to a multiple of 256; a batch for which
+ *     that exceeds NATTN_NOALLOC_SCRATCH_BYTES returns NATTN_ETOOLARGE and
+ *     launches nothing.  Fewer splits than nattn_fwd_ex would use means
+ *     longer runs of pages per CTA: same result, less parallelism.
  *   - The first call on a device looks up that device's address of the
- *     array (cudaGetSymbolAddress, with the device current); make that first
- *     call outside any stream capture.
+ *     array (cudaGetSymbolAddress, with the device current) and keeps it
+ *     with the id of the device's current context; a call that finds a
+ *     different context current (after cudaDeviceReset, say) looks it up
+ *     again.  Make the first call, and the first after such a change,
+ *     outside any stream capture.
  *   - Every call shares the one array and leaves its contents behind.  The
  *     kernels overwrite every partial they later read, so nothing has to
  *     start at zero, but calls that overlap on the GPU (other streams, other

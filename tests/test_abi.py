@@ -114,3 +114,13 @@ def test_workspace_sizes(L):
     assert w0 > 0
     p.normalizer = 3                     # sparse decode also stores scores
     assert L.nattn_workspace_size(p) > w0 + 64 * 32 * 32768 * 4 - 1
+
+
+def test_short_form_paged_needs_device_allocations(L):
+    """nattn_fwd in paged mode bounds the page pool by the device
+    allocations holding k and v; pointers outside any device allocation of
+    this process are refused on the host (NATTN_EINVAL) before any launch."""
+    import ctypes as C
+    rc = L.nattn_fwd(4096, 8192, 12288, 16384, None, 2, 8, 2, 1, 256, 128, 128,
+                     0.088, 0, 1, 0, 0.0, 20480, 24576, None)
+    assert rc == -1

@@ -1,0 +1,188 @@
+"""The contract entry point itself, nattn_fwd, against the float64 oracle.
+
+nattn_fwd takes the backend contract's argument list ("Attention",
+factory.ai transformers wiki, section "What every backend must support";
+the paged cache of "HF Attention Normalizers", section "Differentiable
+Paged Attention") and allocates whatever scratch the chosen path needs
+stream-ordered on the caller's stream.  These tests call it through the C
+ABI with raw device pointers: dense and paged, all four normalizers, ragged
+shapes and one full-size configuration of each mode."""
+
+import numpy as np
+import pytest
+
+from tests._util import (check_out, check_stat, compact_pool, cuda_ok,
+                         ensure_built)
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not cuda_ok(), reason="needs a CUDA device")]
+
+NORMS = ("softmax", "softmax1", "sparsemax", "entmax15")
+NID = {n: i for i, n in enumerate(NORMS)}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    ensure_built()
+
+
+def _call(q, k, v, Tk, normalizer, causal, window=0, softcap=0.0, scale=None,
+          block_table=None, seqlens=None):
+    """nattn_fwd on torch CUDA tensors; returns (rc, out, row_stat)."""
+    import torch
+    from alternative_normalizers_b200 import binding
+    B, Hq, Tq, d = q.shape
+    Hkv, dv = k.shape[1], v.shape[3]
+    out = torch.full((B, Hq, Tq, dv), float("nan"), dtype=torch.bfloat16,
+                     device="cuda")
+    st = torch.full((B, Hq, Tq), float("nan"), dtype=torch.float32,
+                    device="cuda")
+    scale = d ** -0.5 if scale is None else scale
+    stream = torch.cuda.current_stream().cuda_stream
+    rc = binding.nattn_fwd(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), st.data_ptr(),
+        B, Hq, Hkv, Tq, Tk, d, dv, scale, NID[normalizer], int(causal),
+        window, softcap,
+        None if block_table is None else block_table.data_ptr(),
+        None if seqlens is None else seqlens.data_ptr(), stream)
+    torch.cuda.synchronize()
+    return rc, out, st
+
+
+def _rand(g, *shape, gain=1.0):
+    import torch
+    return (torch.randn(*shape, generator=g) * gain).to(torch.bfloat16)
+
+
+DENSE_CASES = [
+    # B, Hq, Hkv, Tq, Tk, d, causal, window, softcap
+    (1, 4, 2, 333, 333, 128, True, 0, 0.0),
+    (2, 3, 1, 150, 270, 64, True, 0, 0.0),      # odd group, Tq != Tk
+    (1, 2, 1, 260, 260, 256, True, 100, 30.0),  # d = 256, window, soft-cap
+    (1, 2, 2, 77, 190, 128, False, 0, 0.0),
+    (1, 2, 1, 45, 45, 40, True, 0, 0.0),        # head dim off the tensor cores
+]
+
+
+@pytest.mark.parametrize("normalizer", NORMS)
+@pytest.mark.parametrize("case", DENSE_CASES, ids=lambda c: "x".join(map(str, c)))
+def test_nattn_fwd_dense(case, normalizer):
+    import torch
+    import oracle
+    from alternative_normalizers_b200 import nattn_get_device_status
+    B, Hq, Hkv, Tq, Tk, d, causal, window, cap = case
+    g = torch.Generator().manual_seed(1234 + Tq + d)
+    q, k, v = _rand(g, B, Hq, Tq, d), _rand(g, B, Hkv, Tk, d), _rand(g, B, Hkv, Tk, d)
+    rc, out, st = _call(q.cuda(), k.cuda(), v.cuda(), Tk, normalizer, causal,
+                        window, cap)
+    assert rc == 0
+    assert nattn_get_device_status() == 0
+    o, s, _ = oracle.attention_fwd(q, k, v, d ** -0.5, normalizer, causal,
+                                   window, cap)
+    check_out(out.float().cpu().numpy(), o, str(case))
+    check_stat(st.cpu().numpy(), s, str(case))
+
+
+def _paged(seed, B, Hq, Hkv, d, lo, hi, Tq=1, spare=0):
+    """Pool of 64-token pages, random permutation, table stride
+    ceil(max_len / 64) (the short form's fixed layout)."""
+    import torch
+    g = torch.Generator().manual_seed(seed)
+    lens = torch.randint(lo, hi + 1, (B,), generator=g)
+    maxlen = int(hi)
+    npg = (lens + 63) // 64
+    P = int(npg.sum()) + spare
+    q = _rand(g, B, Hq, Tq, d)
+    kp = _rand(g, P, Hkv, 64, d)
+    vp = _rand(g, P, Hkv, 64, d)
+    perm = torch.randperm(P, generator=g).to(torch.int32)
+    table = torch.full((B, (maxlen + 63) // 64), -1, dtype=torch.int32)
+    off = 0
+    for b in range(B):
+        table[b, :npg[b]] = perm[off:off + npg[b]]
+        off += int(npg[b])
+    return q, kp, vp, table, lens.to(torch.int32), maxlen
+
+
+@pytest.mark.parametrize("normalizer", NORMS)
+@pytest.mark.parametrize("Tq,group", [(1, 4), (2, 4), (1, 8), (5, 4)])
+def test_nattn_fwd_paged(normalizer, Tq, group):
+    """Paged mode of the short form (64-token pages).  Tq = 5 with a group
+    of 4 is more query rows than the decode kernel takes per CTA, so that
+    case runs on the row-wise kernel."""
+    import torch
+    import oracle
+    from alternative_normalizers_b200 import nattn_get_device_status
+    Hkv = 2
+    q, kp, vp, table, lens, maxlen = _paged(99 + Tq + group, 5, Hkv * group,
+                                            Hkv, 128, 1, 900, Tq, spare=3)
+    rc, out, st = _call(q.cuda(), kp.cuda(), vp.cuda(), maxlen, normalizer,
+                        True, block_table=table.cuda(), seqlens=lens.cuda())
+    assert rc == 0
+    assert nattn_get_device_status() == 0
+    res = oracle.paged_decode(q, kp, vp, table, lens, 64, 128 ** -0.5,
+                              normalizer)
+    for b in range(q.shape[0]):
+        check_out(out[b].float().cpu().numpy(), res[b][0], f"seq {b}")
+        check_stat(st[b].cpu().numpy(), res[b][1], f"seq {b}")
+
+
+def test_nattn_fwd_paged_page_id_past_pool_is_caught():
+    """A page id far past the pool's device allocation is caught on the
+    device (NATTN_EBOUNDS) instead of being read."""
+    import torch
+    from alternative_normalizers_b200 import nattn_get_device_status
+    q, kp, vp, table, lens, maxlen = _paged(7, 3, 8, 2, 128, 100, 400)
+    table[2, 1] = 1 << 24
+    rc, out, st = _call(q.cuda(), kp.cuda(), vp.cuda(), maxlen, "softmax",
+                        True, block_table=table.cuda(), seqlens=lens.cuda())
+    assert rc == 0
+    assert nattn_get_device_status() == -7
+    assert nattn_get_device_status() == 0
+
+
+def test_nattn_fwd_fullsize_dense_sparse():
+    """The sparse prefill workload (B=1, Hq=16, Hkv=8, T=8192, d=128, causal)
+    through nattn_fwd: 1.5-entmax, whose threshold pass and gather need the
+    scratch that nattn_fwd allocates stream-ordered."""
+    import oracle
+    from alternative_normalizers_b200.workloads import WORKLOADS, make_inputs
+    from tests._util import fullsize_rows
+    w = WORKLOADS["sparse_prefill_t1"]
+    x = make_inputs(w)
+    rc, out, st = _call(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(), w.Tk,
+                        "entmax15", True, scale=w.scale)
+    assert rc == 0
+    rows = fullsize_rows(w, 1024)
+    o, s, _ = oracle.attention_rows(x["q"], x["k"], x["v"], rows, w.scale,
+                                    "entmax15", True)
+    out, st = out.float().cpu().numpy(), st.cpu().numpy()
+    check_out(out[rows[:, 0], rows[:, 1], rows[:, 2]], o, "entmax15")
+    check_stat(st[rows[:, 0], rows[:, 1], rows[:, 2]], s, "entmax15")
+    assert np.isfinite(out).all()
+
+
+@pytest.mark.parametrize("normalizer", ("softmax1", "sparsemax"))
+def test_nattn_fwd_fullsize_paged(normalizer):
+    """The paged decode workload (64 sequences, lengths up to 32768,
+    Hq=32, Hkv=8, d=128, 64-token pages) through nattn_fwd."""
+    import oracle
+    from alternative_normalizers_b200.workloads import WORKLOADS, make_inputs
+    w = WORKLOADS["paged_decode"]
+    x = make_inputs(w)
+    assert x["block_table"].shape[1] == (w.len_range[1] + 63) // 64
+    rc, out, st = _call(x["q"].cuda(), x["k_pool"].cuda(), x["v_pool"].cuda(),
+                        w.len_range[1], normalizer, True, scale=w.scale,
+                        block_table=x["block_table"].cuda(),
+                        seqlens=x["seqlens"].cuda())
+    assert rc == 0
+    lens = x["seqlens"].numpy()
+    seqs = sorted({int(np.argmax(lens)), int(np.argmin(lens)), 5, 31})
+    ck, cv, ct = compact_pool(x["k_pool"], x["v_pool"], x["block_table"],
+                              lens, seqs, 64)
+    res = oracle.paged_decode(x["q"], ck, cv, ct, lens, 64, w.scale,
+                              normalizer, seqs=seqs)
+    out, st = out.float().cpu().numpy(), st.cpu().numpy()
+    for b in seqs:
+        check_out(out[b], res[b][0], f"seq {b}")
+        check_stat(st[b], res[b][1], f"seq {b}")

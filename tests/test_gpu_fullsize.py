@@ -1,13 +1,16 @@
 """GPU parity at the full workload sizes, in the launch configuration the
-benchmark times.  The oracle recomputes a seeded sample of query rows one by
-one (first/last rows of tiles, all heads of one KV group, uniform picks);
-the kernels run on the whole problem."""
+benchmark times.  The oracle recomputes at least 1024 seeded query rows per
+workload one by one (tile-edge rows, every head of one KV group, rows at the
+window edge, uniform picks; the same rows on every run); the kernels run on
+the whole problem.  For the sparse normalizers the GPU's support of every
+sampled row (its count of nonzero weights) is checked against the oracle's
+set of keys with p > 0, and the exact-zero fraction is reported."""
 
 import numpy as np
 import pytest
 
-from tests._util import (check_out, check_stat, cuda_ok, ensure_built,
-                         sample_rows)
+from tests._util import (check_out, check_stat, compact_pool, cuda_ok,
+                         ensure_built, fullsize_rows)
 
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not cuda_ok(), reason="needs a CUDA device")]
@@ -30,23 +33,65 @@ def _inputs(name):
     return _cache[name]
 
 
-def _run(w, x, normalizer):
+def _run(w, x, normalizer, want_nnz=False):
     import torch
     from alternative_normalizers_b200 import (attention, nattn_get_device_status,
                                               paged_attention)
+    nnz = None
+    if want_nnz:
+        nnz = torch.full((w.B, w.Hq, w.Tq), -1, dtype=torch.int32, device="cuda")
     if w.paged:
         out, st = paged_attention(
             x["q"].cuda(), x["k_pool"].cuda(), x["v_pool"].cuda(),
             x["block_table"].cuda(), x["seqlens"].cuda(), w.len_range[1],
-            normalizer=normalizer, causal=w.causal)
+            normalizer=normalizer, causal=w.causal, row_nnz=nnz)
     else:
         out, st, _ = attention(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(),
                                normalizer=normalizer, causal=w.causal,
                                window=w.window, softcap=w.softcap,
-                               scale=w.scale)
+                               scale=w.scale, row_nnz=nnz)
     torch.cuda.synchronize()
     assert nattn_get_device_status() == 0
-    return out.float().cpu().numpy(), st.cpu().numpy()
+    return (out.float().cpu().numpy(), st.cpu().numpy(),
+            None if nnz is None else nnz.cpu().numpy())
+
+
+def support_check(w, x, rows, normalizer, tau_o, nnz_gpu):
+    """Compare the GPU's support size of each sampled row with the oracle's
+    set {j : p_j > 0}.  Membership is decided by u_j > tau (u = z for
+    sparsemax, z / 2 for 1.5-entmax); a key within a rounding band of tau
+    may fall on either side, so the GPU count must lie between the oracle's
+    counts at tau + band and tau - band, and equal the oracle's count on
+    every row with no key in the band.  Returns the exact-zero fractions
+    (GPU, oracle) over the visible keys of the sampled rows."""
+    import oracle
+    q = oracle.attention._f64(x["q"])
+    k = oracle.attention._f64(x["k"])
+    group = w.Hq // w.Hkv
+    ok_all = oracle.allowed_matrix(w.Tq, w.Tk, w.causal, w.window)
+    half = 0.5 if normalizer == "entmax15" else 1.0
+    vis = sup_o = sup_g = 0
+    banded = 0
+    for r, (b, h, i) in enumerate(rows):
+        ok = ok_all[i]
+        z = oracle.transform_scores(q[b, h, i] @ k[b, h // group].T, w.scale,
+                                    w.softcap)[ok]
+        u = z * half
+        t = tau_o[r]
+        band = 1e-4 * max(1.0, abs(t))
+        exact = int((u > t).sum())
+        lo, hi = int((u > t + band).sum()), int((u > t - band).sum())
+        g = int(nnz_gpu[r])
+        assert lo <= g <= hi, f"row {(b, h, i)}: gpu {g} oracle [{lo}, {hi}]"
+        if lo == hi:
+            assert g == exact, f"row {(b, h, i)}: gpu {g} oracle {exact}"
+        else:
+            banded += 1
+        vis += ok.sum()
+        sup_o += exact
+        sup_g += g
+    assert banded <= max(2, len(rows) // 100)
+    return 1.0 - sup_g / vis, 1.0 - sup_o / vis
 
 
 DENSE = [("qwen3_8b_prefill", "softmax"), ("qwen3_8b_prefill", "softmax1"),
@@ -60,13 +105,10 @@ DENSE = [("qwen3_8b_prefill", "softmax"), ("qwen3_8b_prefill", "softmax1"),
 def test_fullsize_dense(name, normalizer):
     import oracle
     w, x = _inputs(name)
-    out, st = _run(w, x, normalizer)
-    extra = []
-    if w.window:
-        # rows at the window edge of the local layer
-        extra = [(0, 0, w.window - 1), (0, 0, w.window), (0, 1, w.window + 127)]
-    rows = sample_rows(w.B, w.Hq, w.Tq, 384, seed=hash(name) % 1000,
-                       group=w.Hq // w.Hkv, extra=extra)
+    sparse = normalizer in ("sparsemax", "entmax15")
+    out, st, nnz = _run(w, x, normalizer, want_nnz=sparse)
+    rows = fullsize_rows(w, 1024)
+    assert len(rows) >= 1024
     o, s, _ = oracle.attention_rows(x["q"], x["k"], x["v"], rows, w.scale,
                                     normalizer, w.causal, w.window, w.softcap)
     got_o = out[rows[:, 0], rows[:, 1], rows[:, 2]]
@@ -74,6 +116,12 @@ def test_fullsize_dense(name, normalizer):
     check_out(got_o, o, f"{name}/{normalizer}")
     check_stat(got_s, s, f"{name}/{normalizer}")
     assert np.isfinite(out).all()
+    if sparse:
+        zg, zo = support_check(w, x, rows, normalizer, s,
+                               nnz[rows[:, 0], rows[:, 1], rows[:, 2]])
+        print(f"{name}/{normalizer}: exact-zero fraction gpu {zg:.6f} "
+              f"oracle {zo:.6f} over {len(rows)} rows")
+        assert zg > 0.98 and abs(zg - zo) <= 1e-4
 
 
 def test_fullsize_softmax1_zero_logit_identity():
@@ -98,31 +146,20 @@ def test_fullsize_softmax1_zero_logit_identity():
                                         "entmax15"])
 def test_fullsize_paged_decode(normalizer):
     import oracle
+    from tests._util import workload_seed
     w, x = _inputs("paged_decode")
-    out, st = _run(w, x, normalizer)
-    rng = np.random.default_rng(5)
+    out, st, nnz = _run(w, x, normalizer, want_nnz=True)
+    rng = np.random.default_rng(workload_seed(w.name))
     lens = x["seqlens"].numpy()
     seqs = sorted({int(np.argmax(lens)), int(np.argmin(lens))} |
-                  set(rng.choice(w.B, 4, replace=False).tolist()))
-    res = oracle.paged_decode(x["q"], x["k_pool"], x["v_pool"],
-                              x["block_table"], lens, w.page_size, w.scale,
+                  set(rng.choice(w.B, 6, replace=False).tolist()))
+    ck, cv, ct = compact_pool(x["k_pool"], x["v_pool"], x["block_table"],
+                              lens, seqs, w.page_size)
+    res = oracle.paged_decode(x["q"], ck, cv, ct, lens, w.page_size, w.scale,
                               normalizer, seqs=seqs)
     for b in seqs:
         check_out(out[b], res[b][0], f"seq {b}")
         check_stat(st[b], res[b][1], f"seq {b}")
+        if normalizer in ("softmax", "softmax1"):
+            assert (nnz[b] == lens[b]).all()
     assert np.isfinite(out).all()
-
-
-def test_sparse_exact_zero_fraction_reported():
-    """The sparse normalizers produce exact zeros: on sampled rows of the
-    sparse workload the oracle's zero fraction is high and the GPU's
-    threshold reproduces which keys are in the support."""
-    import oracle
-    w, x = _inputs("sparse_prefill_t4")
-    rows = sample_rows(w.B, w.Hq, w.Tq, 64, seed=3)
-    _, _, wt = oracle.attention_rows(x["q"], x["k"], x["v"], rows, w.scale,
-                                     "sparsemax", True, want_weights=True)
-    ok = np.stack([oracle.allowed_matrix(w.Tq, w.Tk, True, 0)[i]
-                   for i in rows[:, 2]])
-    zero_frac = float(((wt == 0) & ok).sum() / ok.sum())
-    assert zero_frac > 0.99

@@ -141,21 +141,6 @@ def test_tc_sparse_overflow_rows(normalizer):
     check_stat(st, s)
 
 
-@pytest.mark.parametrize("normalizer", ("sparsemax", "entmax15"))
-def test_tc_sparse_apply_on_tensor_cores(normalizer, monkeypatch):
-    """Phase 2 on the tensor cores (NATTN_SPARSE_APPLY=tc): bf16 P from tau
-    times V in a second tcgen05 pass, instead of the fp32 support gather.
-    At the unit query temperature the bf16 weights stay within the output
-    tolerance; tau comes from phase 1 either way."""
-    import oracle
-    monkeypatch.setenv("NATTN_SPARSE_APPLY", "tc")
-    q, k, v = _inputs(21, 1, 4, 2, 448, 448, 128)
-    out, st, _ = _gpu(q, k, v, normalizer=normalizer, causal=True)
-    o, s, _ = oracle.attention_fwd(q, k, v, 128 ** -0.5, normalizer, True)
-    check_out(out, o)
-    check_stat(st, s)
-
-
 def test_softmax1_is_softmax_with_zero_key_on_gpu():
     """GPU softmax1 equals GPU softmax on the input with a zero key and zero
     value prepended (bottom-right causal), which also exercises Tk' = T + 1."""
