@@ -25,6 +25,9 @@ Every function cites the passage of the source pages it restates:
   is_causal; output plus optional weights).
 * "HF Attention Normalizers", section "Packed Variable-Length Attention"
   (bottom-right causal alignment when query and key lengths differ).
+* "Attention variants: what to open up, and how far" (TensorCAD docs),
+  variants table, row "Attention sinks" (a learned per-head term in the
+  softmax's denominator).
 
 Readings where the pages are silent:
 sparsemax is the Euclidean projection onto the probability simplex;
@@ -39,6 +42,7 @@ from .attention import (  # noqa: F401
     transform_scores,
     softmax_row,
     softmax1_row,
+    softmax_sink_row,
     sparsemax_row,
     entmax15_row,
     normalize_row,

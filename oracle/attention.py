@@ -96,6 +96,26 @@ def softmax1_row(z):
     return e / s, m + math.log(s)
 
 
+def softmax_sink_row(z, sink):
+    """softmax with a learned attention sink: ``exp(z_i) / (exp(s) +
+    sum_j exp(z_j))`` for the row's sink logit ``s`` ("Attention variants:
+    what to open up, and how far", TensorCAD, variants table, row "Attention
+    sinks": gpt-oss adds a learned per-head term to the softmax's
+    denominator).  The sink is one more logit whose value row is zero, so
+    this is softmax over ``[z, s]`` with the sink's own weight dropped.
+    ``s = 0`` is softmax1; ``s = -inf`` is plain softmax.  row_stat is
+    ``log(exp(s) + sum exp z)``; an empty row gives no weights and ``s``.
+    """
+    z = np.asarray(z, dtype=np.float64)
+    s = float(sink)
+    m = max(s, float(z.max())) if z.size else s
+    if m == -math.inf:          # no sink and no visible key
+        return z.copy(), -math.inf
+    e = np.exp(z - m)
+    tot = math.exp(s - m) + e.sum()
+    return e / tot, m + math.log(tot)
+
+
 def sparsemax_row(z):
     """sparsemax: Euclidean projection of ``z`` onto the probability simplex
     ("HF Attention Normalizers", "Supported Normalizers": a sparse probability
@@ -176,7 +196,7 @@ def _f64(x):
 
 
 def attention_rows(q, k, v, rows, scale, normalizer, causal=False, window=0,
-                   softcap=0.0, want_weights=False):
+                   softcap=0.0, want_weights=False, sinks=None):
     """Attention output for selected query rows.
 
     ``q`` [B, Hq, Tq, d], ``k`` [B, Hkv, Tk, d], ``v`` [B, Hkv, Tk, dv]
@@ -187,9 +207,16 @@ def attention_rows(q, k, v, rows, scale, normalizer, causal=False, window=0,
     backend must support"), and the reading here is the contiguous grouping
     of that expansion.
 
+    ``sinks`` (length Hq, natural-log logits) turns softmax into softmax
+    with a learned per-head sink (``softmax_sink_row``); only with
+    ``normalizer == "softmax"``.
+
     Returns ``out`` [n, dv], ``row_stat`` [n] and, if asked, dense weights
     [n, Tk] with exact zeros on masked keys.
     """
+    if sinks is not None:
+        assert normalizer == "softmax", "sinks go with softmax"
+        sinks = np.asarray(_f64(sinks), dtype=np.float64).reshape(-1)
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, Hq, Tq, d = q.shape
     _, Hkv, Tk, _ = k.shape
@@ -212,7 +239,10 @@ def attention_rows(q, k, v, rows, scale, normalizer, causal=False, window=0,
         z = transform_scores(s, scale, softcap)
         for t, (r, i) in enumerate(zip(sel, qi)):
             ok = ok_all[i]
-            p, st = normalize_row(z[t][ok], normalizer)
+            if sinks is None:
+                p, st = normalize_row(z[t][ok], normalizer)
+            else:
+                p, st = softmax_sink_row(z[t][ok], sinks[h])
             stat[r] = st
             if p.size:
                 out[r] = p @ v[b, g][ok]
@@ -222,7 +252,7 @@ def attention_rows(q, k, v, rows, scale, normalizer, causal=False, window=0,
 
 
 def attention_fwd(q, k, v, scale, normalizer, causal=False, window=0,
-                  softcap=0.0, want_weights=False):
+                  softcap=0.0, want_weights=False, sinks=None):
     """Full attention forward: ``out`` [B, Hq, Tq, dv], ``row_stat``
     [B, Hq, Tq] and optionally ``weights`` [B, Hq, Tq, Tk] (float64)."""
     qa = _f64(q)
@@ -232,7 +262,7 @@ def attention_fwd(q, k, v, scale, normalizer, causal=False, window=0,
                              indexing="ij")
     rows = np.stack([bb.ravel(), hh.ravel(), ii.ravel()], axis=1)
     out, stat, w = attention_rows(qa, k, v, rows, scale, normalizer, causal,
-                                  window, softcap, want_weights)
+                                  window, softcap, want_weights, sinks)
     dv = out.shape[1]
     out = out.reshape(B, Hq, Tq, dv)
     stat = stat.reshape(B, Hq, Tq)
@@ -269,7 +299,8 @@ def paged_gather(k_pool, v_pool, block_table, seqlen, b, page_size):
 
 
 def paged_decode(q, k_pool, v_pool, block_table, seqlens, page_size, scale,
-                 normalizer, causal=True, window=0, softcap=0.0, seqs=None):
+                 normalizer, causal=True, window=0, softcap=0.0, seqs=None,
+                 sinks=None):
     """Attention of ``q`` [B, Hq, Tq, d] over each sequence's paged K/V.
 
     Each sequence has its own key length ``seqlens[b]``; the query rows are
@@ -285,6 +316,7 @@ def paged_decode(q, k_pool, v_pool, block_table, seqlens, page_size, scale,
         kk, vv = paged_gather(k_pool, v_pool, block_table, int(lens[b]), b,
                               page_size)
         o, st, _ = attention_fwd(qa[b:b + 1], kk[None], vv[None], scale,
-                                 normalizer, causal, window, softcap)
+                                 normalizer, causal, window, softcap,
+                                 sinks=sinks)
         res[int(b)] = (o[0], st[0])
     return res
