@@ -25,6 +25,9 @@ Every function cites the passage of the source pages it restates:
   is_causal; output plus optional weights).
 * "HF Attention Normalizers", section "Packed Variable-Length Attention"
   (bottom-right causal alignment when query and key lengths differ).
+* "HF Attention Normalizers", section "Important Limitations" for the
+  backward pass (saved row statistics, probabilities recomputed; gradients
+  in ``backward.py``).
 * "Attention variants: what to open up, and how far" (TensorCAD docs),
   variants table, row "Attention sinks" (a learned per-head term in the
   softmax's denominator).
@@ -51,3 +54,4 @@ from .attention import (  # noqa: F401
     paged_gather,
     paged_decode,
 )
+from .backward import attention_bwd, row_vjp  # noqa: F401
