@@ -39,6 +39,26 @@ class NattnArgs(ctypes.Structure):
         ("page_size", ctypes.c_int), ("block_table_stride", ctypes.c_int),
         ("num_pages", ctypes.c_int),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("stream", ctypes.c_void_p), ("sinks", ctypes.c_void_p),
+    ]
+
+
+class NattnBwdArgs(ctypes.Structure):
+    """Mirror of ``nattn_bwd_args``."""
+
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("out", ctypes.c_void_p), ("grad_out", ctypes.c_void_p),
+        ("row_stat", ctypes.c_void_p),
+        ("grad_q", ctypes.c_void_p), ("grad_k", ctypes.c_void_p),
+        ("grad_v", ctypes.c_void_p),
+        ("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+        ("Tq", ctypes.c_int), ("Tk", ctypes.c_int), ("d", ctypes.c_int),
+        ("dv", ctypes.c_int),
+        ("scale", ctypes.c_float), ("normalizer", ctypes.c_int),
+        ("causal", ctypes.c_int), ("window", ctypes.c_int),
+        ("softcap", ctypes.c_float), ("sinks", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("stream", ctypes.c_void_p),
     ]
 
@@ -81,6 +101,11 @@ def lib():
         L.nattn_version.restype = ctypes.c_int
         L.nattn_decode_noalloc.argtypes = [P]
         L.nattn_decode_noalloc.restype = ctypes.c_int
+        PB = ctypes.POINTER(NattnBwdArgs)
+        L.nattn_bwd.argtypes = [PB]
+        L.nattn_bwd.restype = ctypes.c_int
+        L.nattn_bwd_workspace_size.argtypes = [PB]
+        L.nattn_bwd_workspace_size.restype = ctypes.c_size_t
         L.nattn_selftest_wait_timeout.argtypes = [ctypes.c_void_p]
         L.nattn_selftest_wait_timeout.restype = ctypes.c_int
         _lib = L
@@ -106,6 +131,14 @@ def nattn_fwd_ex(args: NattnArgs):
 
 def nattn_workspace_size(args: NattnArgs):
     return lib().nattn_workspace_size(ctypes.byref(args))
+
+
+def nattn_bwd(args: NattnBwdArgs):
+    return lib().nattn_bwd(ctypes.byref(args))
+
+
+def nattn_bwd_workspace_size(args: NattnBwdArgs):
+    return lib().nattn_bwd_workspace_size(ctypes.byref(args))
 
 
 def nattn_get_device_status(stream=None):
@@ -149,16 +182,18 @@ def _norm_id(normalizer):
 def build_args(q, k, v, out, row_stat=None, weights=None, *, normalizer,
                causal=False, window=0, softcap=0.0, scale=None,
                block_table=None, seqlens=None, page_size=0, max_seqlen=None,
-               stream=None, row_nnz=None):
+               stream=None, row_nnz=None, sinks=None):
     """Fill an ``NattnArgs`` from torch tensors (no device work).
     ``row_nnz`` (int32 [B, Hq, Tq] or None) receives the number of keys with
-    a nonzero weight in each row."""
+    a nonzero weight in each row; ``sinks`` (float32 [Hq] or None) are the
+    learned per-head sink logits (softmax only)."""
     import torch
     B, Hq, Tq, d = q.shape
     a = NattnArgs()
     a.q, a.k, a.v, a.out = _ptr(q), _ptr(k), _ptr(v), _ptr(out)
     a.row_stat, a.weights = _ptr(row_stat), _ptr(weights)
     a.row_nnz = _ptr(row_nnz)
+    a.sinks = _ptr(sinks)
     a.B, a.Hq, a.Tq, a.d = B, Hq, Tq, d
     a.Hkv = k.shape[1]
     a.dv = v.shape[3]
@@ -194,10 +229,11 @@ def _run(a, workspace_holder):
 
 def attention(q, k, v, normalizer="softmax", causal=False, window=0,
               softcap=0.0, scale=None, want_weights=False, out=None,
-              row_stat=None, row_nnz=None):
+              row_stat=None, row_nnz=None, sinks=None):
     """Dense attention forward.  q [B,Hq,Tq,d], k [B,Hkv,Tk,d], v
     [B,Hkv,Tk,dv] (bf16, CUDA, contiguous).  Returns (out, row_stat,
-    weights|None); fills ``row_nnz`` (int32 [B,Hq,Tq]) when given."""
+    weights|None); fills ``row_nnz`` (int32 [B,Hq,Tq]) when given.
+    ``sinks`` (float32 [Hq], softmax only): learned per-head sink logits."""
     import torch
     B, Hq, Tq, _ = q.shape
     Tk, dv = k.shape[2], v.shape[3]
@@ -209,7 +245,7 @@ def attention(q, k, v, normalizer="softmax", causal=False, window=0,
                           device=q.device) if want_weights else None
     a = build_args(q, k, v, out, row_stat, weights, normalizer=normalizer,
                    causal=causal, window=window, softcap=softcap, scale=scale,
-                   row_nnz=row_nnz)
+                   row_nnz=row_nnz, sinks=sinks)
     keep = []
     _run(a, keep)
     return out, row_stat, weights
@@ -217,7 +253,8 @@ def attention(q, k, v, normalizer="softmax", causal=False, window=0,
 
 def paged_attention(q, k_pool, v_pool, block_table, seqlens, max_seqlen,
                     normalizer="softmax", causal=True, window=0, softcap=0.0,
-                    scale=None, out=None, row_stat=None, row_nnz=None):
+                    scale=None, out=None, row_stat=None, row_nnz=None,
+                    sinks=None):
     """Attention of q [B,Hq,Tq,d] over a paged cache: k_pool/v_pool
     [num_pages, Hkv, page, d], block_table int32 [B, max_pages], seqlens
     int32 [B] (each <= max_seqlen).  Fills ``row_nnz`` when given."""
@@ -232,7 +269,49 @@ def paged_attention(q, k_pool, v_pool, block_table, seqlens, max_seqlen,
                    normalizer=normalizer, causal=causal, window=window,
                    softcap=softcap, scale=scale, block_table=block_table,
                    seqlens=seqlens, page_size=k_pool.shape[2],
-                   max_seqlen=max_seqlen, row_nnz=row_nnz)
+                   max_seqlen=max_seqlen, row_nnz=row_nnz, sinks=sinks)
     keep = []
     _run(a, keep)
     return out, row_stat
+
+
+def build_bwd_args(q, k, v, out, row_stat, grad_out, grad_q, grad_k, grad_v, *,
+                   normalizer, causal=False, window=0, softcap=0.0,
+                   scale=None, sinks=None, stream=None):
+    """Fill an ``NattnBwdArgs`` from torch tensors (no device work)."""
+    import torch
+    B, Hq, Tq, d = q.shape
+    a = NattnBwdArgs()
+    a.q, a.k, a.v, a.out = _ptr(q), _ptr(k), _ptr(v), _ptr(out)
+    a.grad_out, a.row_stat = _ptr(grad_out), _ptr(row_stat)
+    a.grad_q, a.grad_k, a.grad_v = _ptr(grad_q), _ptr(grad_k), _ptr(grad_v)
+    a.B, a.Hq, a.Tq, a.d = B, Hq, Tq, d
+    a.Hkv, a.Tk, a.dv = k.shape[1], k.shape[2], v.shape[3]
+    a.scale = (1.0 / d ** 0.5) if scale is None else scale
+    a.normalizer = _norm_id(normalizer)
+    a.causal, a.window, a.softcap = int(bool(causal)), int(window), float(softcap)
+    a.sinks = _ptr(sinks)
+    if stream is None and q.is_cuda:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    a.stream = stream
+    return a
+
+
+def attention_backward(q, k, v, out, row_stat, grad_out, normalizer="softmax",
+                       causal=False, window=0, softcap=0.0, scale=None,
+                       sinks=None):
+    """Gradients (dq, dk, dv) of sum(grad_out * O) for the dense forward
+    that produced ``out`` and ``row_stat`` with the same arguments (bf16,
+    CUDA, contiguous; d == dv in {64, 128})."""
+    import torch
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    a = build_bwd_args(q, k, v, out, row_stat, grad_out, dq, dk, dv,
+                       normalizer=normalizer, causal=causal, window=window,
+                       softcap=softcap, scale=scale, sinks=sinks)
+    need = nattn_bwd_workspace_size(a)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    a.workspace, a.workspace_bytes = ws.data_ptr(), need
+    rc = nattn_bwd(a)
+    if rc != NATTN_OK:
+        raise NattnError(rc, "nattn_bwd")
+    return dq, dk, dv

@@ -57,6 +57,20 @@ __device__ __forceinline__ float fast_exp2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// p_k = 2^(r_k * fa - m) for 64 scores held as raw bits; returns the bf16
+// pairs packed for a TMEM store and adds the fp32 weights into s0 / s1.
+__device__ __forceinline__ void exp2_pack64(const uint32_t* r, float fa, float m, float& s0,
+                                            float& s1, uint32_t (&pk)[32]) {
+#pragma unroll
+  for (int k = 0; k < 64; k += 2) {
+    const float p0 = fast_exp2(fmaf(__uint_as_float(r[k]), fa, -m));
+    const float p1 = fast_exp2(fmaf(__uint_as_float(r[k + 1]), fa, -m));
+    s0 += p0;
+    s1 += p1;
+    pk[k >> 1] = pack_bf16(p0, p1);
+  }
+}
+
 __device__ __forceinline__ float fast_tanh(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -242,6 +256,19 @@ __device__ __forceinline__ void umma_ts(uint32_t d, uint32_t a_tmem, uint64_t bd
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accum)
       : "memory");
 }
+// Re-split the block's registers between warpgroups: every warp of the
+// warpgroup executes the same one (a warpgroup that lowers its count returns
+// registers to the block's pool, one that raises it waits until the pool has
+// them).
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Arrive on an mbarrier once every tcgen05 op issued so far by this thread
 // has completed.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {

@@ -433,7 +433,8 @@ __global__ void __launch_bounds__(DEC_THREADS)
 }
 
 // Merge the splits of every query row.  ONLINE: rescale each split's (m, l, O)
-// to the common maximum; softmax1 adds its logit-0 sink exactly once here.
+// to the common maximum; the sink (softmax1's logit 0 or a learned per-head
+// logit) is added exactly once here.
 // APPLY: plain sum of the partial outputs; row_stat = tau.
 __global__ void decode_combine_kernel(DecodeArgs A, int mode) {
   const Problem& P = A.P;
@@ -449,10 +450,12 @@ __global__ void decode_combine_kernel(DecodeArgs A, int mode) {
   const int nact = min(A.nsplit, (npages + A.pps - 1) / A.pps);
   const size_t pbase = (((size_t)b * P.Hkv + g) * A.nsplit) * A.R + r;
   if (mode == DEC_ONLINE) {
-    float M = (P.norm == NATTN_SOFTMAX1) ? 0.f : -INFINITY;
+    // the sink (softmax1: logit 0; learned per-head sink) enters once, here
+    const float sink2 = sink_logit(P, h) * 1.4426950408889634f;
+    float M = sink2;
     for (int s = 0; s < nact; ++s) M = fmaxf(M, A.ml[(pbase + (size_t)s * A.R) * 2]);
     const float msafe = (M == -INFINITY) ? 0.f : M;
-    float l = (P.norm == NATTN_SOFTMAX1) ? fast_exp2(-msafe) : 0.f;
+    float l = (sink2 == -INFINITY) ? 0.f : fast_exp2(sink2 - msafe);
     for (int s = 0; s < nact; ++s) {
       const float ms = A.ml[(pbase + (size_t)s * A.R) * 2];
       l += A.ml[(pbase + (size_t)s * A.R) * 2 + 1] * fast_exp2(ms - msafe);

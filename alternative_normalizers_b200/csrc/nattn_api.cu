@@ -12,6 +12,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include "backward.cuh"
 #include "common.cuh"
 #include "decode.cuh"
 #include "prefill_pair.cuh"
@@ -157,8 +158,10 @@ int validate(const nattn_args* a) {
     return NATTN_EALIGN;
   if ((a->row_stat && (reinterpret_cast<uintptr_t>(a->row_stat) & 3)) ||
       (a->weights && (reinterpret_cast<uintptr_t>(a->weights) & 3)) ||
-      (a->row_nnz && (reinterpret_cast<uintptr_t>(a->row_nnz) & 3)))
+      (a->row_nnz && (reinterpret_cast<uintptr_t>(a->row_nnz) & 3)) ||
+      (a->sinks && (reinterpret_cast<uintptr_t>(a->sinks) & 3)))
     return NATTN_EALIGN;
+  if (a->sinks && a->normalizer != NATTN_SOFTMAX) return NATTN_EUNSUPPORTED;
   const long long rows = (long long)a->B * a->Hq * a->Tq;
   if (rows >= (1ll << 31) || rows * (long long)(a->d > a->dv ? a->d : a->dv) >= (1ll << 40))
     return NATTN_ETOOLARGE;
@@ -276,6 +279,7 @@ Problem to_problem(const nattn_args* a) {
   P.causal = a->causal;
   P.window = a->window;
   P.softcap = a->softcap;
+  P.sinks = a->sinks;
   P.block_table = a->block_table;
   P.seqlens = a->seqlens;
   P.page_size = a->page_size;
@@ -329,7 +333,9 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
     if constexpr (D <= 128) {
       if ((a->Hq / a->Hkv) % 2 == 0) {
         using PL = PairLayout<D, KST, VST>;
-        auto kp = prefill_pair_kernel<D, KST, VST>;
+        const bool cap = a->softcap > 0.f || !(A.zscale > 0.f);
+        auto kp = cap ? prefill_pair_kernel<D, KST, VST, true>
+                      : prefill_pair_kernel<D, KST, VST, false>;
         if (allow_smem(kp, PL::ALLOC) != cudaSuccess) return NATTN_ECUDA;
         const unsigned pgrid = (unsigned)((long long)a->B * (a->Hq / 2) * ntq);
         kp<<<pgrid, PAIR_THREADS, PL::ALLOC, st>>>(mq, mk, mv, A);
@@ -564,6 +570,126 @@ int decode_noalloc(const nattn_args* a) {
   return launch_decode<256, 64>(a, P, pl, ws, st);
 }
 
+// ---------------------------------------------------------------------------
+// Backward
+// ---------------------------------------------------------------------------
+int validate_bwd(const nattn_bwd_args* a) {
+  if (a == nullptr) return NATTN_EINVAL;
+  nattn_args f;
+  memset(&f, 0, sizeof(f));
+  f.q = a->q;
+  f.k = a->k;
+  f.v = a->v;
+  f.out = a->grad_q;  // any non-null output pointer for the shared checks
+  f.B = a->B;
+  f.Hq = a->Hq;
+  f.Hkv = a->Hkv;
+  f.Tq = a->Tq;
+  f.Tk = a->Tk;
+  f.d = a->d;
+  f.dv = a->dv;
+  f.scale = a->scale;
+  f.normalizer = a->normalizer;
+  f.causal = a->causal;
+  f.window = a->window;
+  f.softcap = a->softcap;
+  f.sinks = a->sinks;
+  f.row_stat = const_cast<float*>(a->row_stat);
+  int rc = validate(&f);
+  if (rc != NATTN_OK) return rc;
+  if (a->B == 0 || a->Hq == 0 || a->Tq == 0) return NATTN_OK;
+  if (!a->out || !a->grad_out || !a->row_stat || !a->grad_q || !a->grad_k || !a->grad_v)
+    return NATTN_EINVAL;
+  if (!aligned16(a->out) || !aligned16(a->grad_out) || !aligned16(a->grad_q) ||
+      !aligned16(a->grad_k) || !aligned16(a->grad_v))
+    return NATTN_EALIGN;
+  if (a->d != a->dv || (a->d != 64 && a->d != 128) || a->Tk < 1) return NATTN_EUNSUPPORTED;
+  return NATTN_OK;
+}
+
+size_t bwd_workspace(const nattn_bwd_args* a) {
+  return up256((size_t)a->B * a->Hq * a->Tq * 4);
+}
+
+template <int D>
+int launch_bwd(const nattn_bwd_args* a, cudaStream_t st) {
+  BwdArgs A;
+  memset(&A, 0, sizeof(A));
+  Problem& P = A.P;
+  P.q = static_cast<const bf16*>(a->q);
+  P.k = static_cast<const bf16*>(a->k);
+  P.v = static_cast<const bf16*>(a->v);
+  P.out = static_cast<bf16*>(const_cast<void*>(a->out));
+  P.row_stat = const_cast<float*>(a->row_stat);
+  P.B = a->B;
+  P.Hq = a->Hq;
+  P.Hkv = a->Hkv;
+  P.Tq = a->Tq;
+  P.Tk = a->Tk;
+  P.d = a->d;
+  P.dv = a->dv;
+  P.scale = a->scale;
+  P.norm = a->normalizer;
+  P.causal = a->causal;
+  P.window = a->window;
+  P.softcap = a->softcap;
+  P.sinks = a->sinks;
+  A.dout = static_cast<const bf16*>(a->grad_out);
+  A.dq = static_cast<bf16*>(a->grad_q);
+  A.dk = static_cast<bf16*>(a->grad_k);
+  A.dv = static_cast<bf16*>(a->grad_v);
+  A.delta = static_cast<float*>(a->workspace);
+  A.us = (a->normalizer == NATTN_ENTMAX15) ? 0.5f : 1.0f;
+  const bool sparse = a->normalizer == NATTN_SPARSEMAX || a->normalizer == NATTN_ENTMAX15;
+  const long long BHq = (long long)a->B * a->Hq, BHkv = (long long)a->B * a->Hkv;
+  // dQ kernel: 128-row query tiles, 64-key blocks
+  CUtensorMap mq, mo, mk, mv;
+  if (!make_map_3d(&mq, a->q, D, a->Tq, BHq, 128) ||
+      !make_map_3d(&mo, a->grad_out, D, a->Tq, BHq, 128) ||
+      !make_map_3d(&mk, a->k, D, a->Tk, BHkv, BWD_BN) ||
+      !make_map_3d(&mv, a->v, D, a->Tk, BHkv, BWD_BN))
+    return NATTN_ECUDA;
+  const unsigned gq = (unsigned)(BHq * ((a->Tq + 127) / 128));
+  using LQ = BwdQLayout<D, D>;
+  if (sparse) {
+    auto k = bwd_dq_kernel<D, D, BWD_DELTA>;
+    if (allow_smem(k, LQ::ALLOC) != cudaSuccess) return NATTN_ECUDA;
+    k<<<gq, BWD_THREADS, LQ::ALLOC, st>>>(mq, mo, mk, mv, A);
+  } else {
+    const size_t rows = (size_t)BHq * a->Tq;
+    bwd_delta_dot_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(A);
+  }
+  if (check_launch() != NATTN_OK) return NATTN_ECUDA;
+  {
+    auto k = bwd_dq_kernel<D, D, BWD_DQ>;
+    if (allow_smem(k, LQ::ALLOC) != cudaSuccess) return NATTN_ECUDA;
+    k<<<gq, BWD_THREADS, LQ::ALLOC, st>>>(mq, mo, mk, mv, A);
+    if (check_launch() != NATTN_OK) return NATTN_ECUDA;
+  }
+  // dK/dV kernel: 128-key tiles, 64-row query blocks
+  if (!make_map_3d(&mq, a->q, D, a->Tq, BHq, BWD_BQ) ||
+      !make_map_3d(&mo, a->grad_out, D, a->Tq, BHq, BWD_BQ) ||
+      !make_map_3d(&mk, a->k, D, a->Tk, BHkv, 128) ||
+      !make_map_3d(&mv, a->v, D, a->Tk, BHkv, 128))
+    return NATTN_ECUDA;
+  using LK = BwdKVLayout<D, D>;
+  auto k = bwd_dkdv_kernel<D, D>;
+  if (allow_smem(k, LK::ALLOC) != cudaSuccess) return NATTN_ECUDA;
+  const unsigned gk = (unsigned)(BHkv * ((a->Tk + 127) / 128));
+  k<<<gk, BWD_THREADS, LK::ALLOC, st>>>(mq, mo, mk, mv, A);
+  return check_launch();
+}
+
+int run_bwd(const nattn_bwd_args* a) {
+  int rc = validate_bwd(a);
+  if (rc != NATTN_OK) return rc;
+  if (a->B == 0 || a->Hq == 0 || a->Tq == 0) return NATTN_OK;
+  if (a->workspace == nullptr || a->workspace_bytes < bwd_workspace(a)) return NATTN_EWORKSPACE;
+  if (!aligned16(a->workspace)) return NATTN_EALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(a->stream);
+  return a->d == 64 ? launch_bwd<64>(a, st) : launch_bwd<128>(a, st);
+}
+
 }  // namespace
 
 namespace nattn {
@@ -587,6 +713,16 @@ __global__ void selftest_wait_kernel() {
 extern "C" {
 
 __attribute__((visibility("default"))) int nattn_fwd_ex(const nattn_args* a) { return run(a); }
+
+__attribute__((visibility("default"))) int nattn_bwd(const nattn_bwd_args* a) {
+  return run_bwd(a);
+}
+
+__attribute__((visibility("default"))) size_t nattn_bwd_workspace_size(const nattn_bwd_args* a) {
+  if (validate_bwd(a) != NATTN_OK) return 0;
+  if (a->B == 0 || a->Hq == 0 || a->Tq == 0) return 0;
+  return bwd_workspace(a);
+}
 
 __attribute__((visibility("default"))) size_t nattn_workspace_size(const nattn_args* a) {
   if (validate(a) != NATTN_OK) return 0;

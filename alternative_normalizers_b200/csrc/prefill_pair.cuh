@@ -26,7 +26,16 @@
 
 namespace nattn {
 
-constexpr int PAIR_THREADS = 320;  // 8 normalizer warps + TMA warp + MMA warp
+// 12 warps: two normalizer warpgroups (warps 0-7), then a third warpgroup
+// with the TMA warp (8), the MMA warp (9) and two warps with no role.  The
+// block is launched at 168 registers a thread (384 x 168 = 64512); the third
+// warpgroup gives back down to 56 and the normalizer warpgroups take 224,
+// enough to hold a whole S row: 2 x 128 x 224 + 128 x 56 = 64512.
+constexpr int PAIR_THREADS = 384;
+constexpr int PAIR_REGS_NORM = 224;
+constexpr int PAIR_REGS_CTRL = 56;
+static_assert(2 * 128 * PAIR_REGS_NORM + 128 * PAIR_REGS_CTRL <= PAIR_THREADS * 168,
+              "register split exceeds the launch allocation");
 
 template <int D, int KST, int VST>
 struct PairLayout {
@@ -51,10 +60,9 @@ struct PairLayout {
 };
 
 // One normalizer warp of tile t = warp / 4: thread = query row = TMEM lane of
-// its lane quarter.  The S row is read in two 64-column halves twice (maximum,
-// then exponentials), which keeps the register count within the 320-thread
-// budget; TMEM reads are cheap next to the exponentials.
-template <int D, int KST, int VST>
+// its lane quarter.  The S row is read from TMEM once per block and held in
+// registers (128 values) for the maximum and the exponentials.
+template <int D, int KST, int VST, bool CAP>
 __device__ __forceinline__ void prefill_pair_normalizer(
     const TcArgs& A, uint8_t* smem, uint32_t tmem, int warp, int lane, int q0, int bh0,
     int kb0, int nblk, uint32_t bar_sf, uint32_t bar_pf, uint32_t bar_pvt,
@@ -73,11 +81,15 @@ __device__ __forceinline__ void prefill_pair_normalizer(
   const uint32_t sbase = lane_base + LY::TM_S + t * BN;
   const uint32_t obase = lane_base + LY::TM_O + t * D;
   const size_t flat = (size_t)(bh0 + t) * P.Tq + qi;
-  const bool fast = !(P.softcap > 0.f) && A.zscale > 0.f;
+  // CAP: soft-cap (or a non-positive scale), scores go through tc_z; else
+  // max(z) = scale * max(s) and exp2(z - m) is one FFMA + EX2 per score
+  constexpr bool fast = !CAP;
   const float fa = fast ? A.zscale : 1.f;  // p = exp2(x * fa - m)
-  const bool sm1 = P.norm == NATTN_SOFTMAX1;
-  float m_run = sm1 ? 0.f : -INFINITY;
-  float l_run = sm1 ? 1.f : 0.f;
+  // the running state starts from the sink (softmax1: logit 0; a learned
+  // per-head sink: its logit, here in log2 units): m0 = sink, l0 = 1
+  const float sink2 = sink_logit(P, (bh0 + t) % P.Hq) * 1.4426950408889634f;
+  float m_run = sink2;
+  float l_run = (sink2 == -INFINITY) ? 0.f : 1.f;
   bool alive = true;
 
   for (int j = 0; j < nblk; ++j) {
@@ -94,37 +106,25 @@ __device__ __forceinline__ void prefill_pair_normalizer(
       kl = BN;
       span = 0;
     }
-    // scores of one 64-column half -> x (raw on the fast path, else z in
-    // log2 units), masked entries -inf
-    auto load_half = [&](int hh, uint32_t (&r)[64]) {
-      tmem_ld32(sbase + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-      tmem_ld32(sbase + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-      tmem_ld_wait();
-      if (!fast) {
+    // the whole S row (128 scores) in registers: one TMEM read per block;
+    // x is the raw score on the fast path, else z in log2 units; masked
+    // entries -inf
+    uint32_t r[BN];
 #pragma unroll
-        for (int k = 0; k < 64; ++k) r[k] = __float_as_uint(tc_z(__uint_as_float(r[k]), A));
-      }
-      if (edge) {
+    for (int c = 0; c < BN / 32; ++c)
+      tmem_ld32(sbase + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+    tmem_ld_wait();
+    if (!fast) {
 #pragma unroll
-        for (int k = 0; k < 64; ++k)
-          if ((unsigned)(hh * 64 + k - kl) > span) r[k] = __float_as_uint(-INFINITY);
-      }
-    };
-    float mx = -INFINITY;
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      uint32_t r[64];
-      load_half(hh, r);
-      float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
-#pragma unroll
-      for (int k = 0; k < 64; k += 4) {
-        a0 = fmaxf(a0, __uint_as_float(r[k]));
-        a1 = fmaxf(a1, __uint_as_float(r[k + 1]));
-        a2 = fmaxf(a2, __uint_as_float(r[k + 2]));
-        a3 = fmaxf(a3, __uint_as_float(r[k + 3]));
-      }
-      mx = fmaxf(mx, fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)));
+      for (int k = 0; k < BN; ++k) r[k] = __float_as_uint(tc_z(__uint_as_float(r[k]), A));
     }
+    if (edge) {
+#pragma unroll
+      for (int k = 0; k < BN; ++k)
+        if ((unsigned)(k - kl) > span) r[k] = __float_as_uint(-INFINITY);
+    }
+    float mx = fmaxf(fmaxf(max32_bits(&r[0]), max32_bits(&r[32])),
+                     fmaxf(max32_bits(&r[64]), max32_bits(&r[96])));
     mx *= fa;
     const float mnew = fmaxf(m_run, mx);
     const bool resc = mnew > m_run + 8.f;  // move the maximum only when it grows by 2^8
@@ -134,17 +134,8 @@ __device__ __forceinline__ void prefill_pair_normalizer(
     float s0 = 0.f, s1 = 0.f;
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
-      uint32_t r[64];
-      load_half(hh, r);
       uint32_t pk[32];
-#pragma unroll
-      for (int k = 0; k < 64; k += 2) {
-        const float p0 = fast_exp2(fmaf(__uint_as_float(r[k]), fa, -msafe));
-        const float p1 = fast_exp2(fmaf(__uint_as_float(r[k + 1]), fa, -msafe));
-        s0 += p0;
-        s1 += p1;
-        pk[k >> 1] = pack_bf16(p0, p1);
-      }
+      exp2_pack64(&r[hh * 64], fa, msafe, s0, s1, pk);
       // packed P of keys [64 hh, 64 hh + 64) over S columns already read
       tmem_st32(sbase + hh * 32, pk);
     }
@@ -208,7 +199,7 @@ __device__ __forceinline__ void prefill_pair_normalizer(
   if (row_ok && P.row_nnz) P.row_nnz[flat] = rr.hi >= rr.lo ? rr.hi - rr.lo + 1 : 0;
 }
 
-template <int D, int KST, int VST>
+template <int D, int KST, int VST, bool CAP>
 __global__ void __launch_bounds__(PAIR_THREADS, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq,
                         const __grid_constant__ CUtensorMap tmk,
@@ -280,108 +271,113 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = misc[0];
 
-  if (warp == 8) {
-    // ======================= TMA producer ===================================
-    if (lane == 0 && nblk > 0) {
-      tma_prefetch_desc(&tmq);
-      tma_prefetch_desc(&tmk);
-      tma_prefetch_desc(&tmv);
-      mbar_expect_tx(bar_q, 2 * LY::QBYTES);
-#pragma unroll
-      for (int t = 0; t < 2; ++t)
-#pragma unroll
-        for (int x = 0; x < D / 64; ++x)
-          tma_load_3d(smem_addr(smem + LY::OFF_Q + t * LY::QBYTES + x * TC_BM * 128), &tmq,
-                      bar_q, x * 64, q0, bh0 + t);
-      for (int j = 0; j < nblk; ++j) {
-        const int kb = kb0 + j;
-        const int ks = j % KST;
-        if (j >= KST && !mbar_wait(bar_kempty(ks), ((j / KST) + 1) & 1, abort_flag)) break;
-        mbar_expect_tx(bar_kfull(ks), LY::KBYTES);
-        uint8_t* kdst = smem + LY::OFF_K + ks * LY::KBYTES;
-#pragma unroll
-        for (int x = 0; x < D / 64; ++x)
-          tma_load_3d(smem_addr(kdst + x * BN * 128), &tmk, bar_kfull(ks), x * 64, kb * BN,
-                      b * P.Hkv + g);
-        const int vs = j % VST;
-        if (j >= VST && !mbar_wait(bar_vempty(vs), ((j / VST) + 1) & 1, abort_flag)) break;
-        mbar_expect_tx(bar_vfull(vs), LY::VBYTES);
-        uint8_t* vdst = smem + LY::OFF_V + vs * LY::VBYTES;
-#pragma unroll
-        for (int x = 0; x < D / 64; ++x)
-          tma_load_3d(smem_addr(vdst + x * BN * 128), &tmv, bar_vfull(vs), x * 64, kb * BN,
-                      b * P.Hkv + g);
-      }
-    }
-  } else if (warp == 9) {
-    // ======================= MMA issuer =====================================
-    if (lane == 0 && nblk > 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16(TC_BM, BN, 0, 0);
-      constexpr uint32_t IDESC_O = idesc_bf16(TC_BM, D, 0, 1);
-      bool ok = mbar_wait_spin(bar_q, 0, abort_flag);
-      tc_fence_after();
-      auto issue_qk = [&](int t, int j) {
-        const uint32_t qbase = smem_addr(smem + LY::OFF_Q + t * LY::QBYTES);
-        const uint32_t kbase = smem_addr(smem + LY::OFF_K + (j % KST) * LY::KBYTES);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad =
-              sdesc_sw128(qbase + (kk >> 2) * TC_BM * 128 + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(kbase + (kk >> 2) * BN * 128 + (kk & 3) * 32, 16, 1024);
-          umma_ss(tmem + LY::TM_S + t * BN, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(bar_sfull(t));
-      };
-      // prologue: both tiles' scores of the first block
-      if (ok && mbar_wait_spin(bar_kfull(0), 0, abort_flag)) {
-        tc_fence_after();
-        issue_qk(0, 0);
-        issue_qk(1, 0);
-        umma_commit(bar_kempty(0));
-      } else {
-        ok = false;
-      }
-      for (int j = 0; ok && j < nblk; ++j) {
-        const int vs = j % VST;
-        if (!mbar_wait_spin(bar_vfull(vs), (j / VST) & 1, abort_flag)) break;
-        bool k_next = false;
-        for (int t = 0; t < 2; ++t) {
-          if (!mbar_wait_spin(bar_pfull(t), j & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t vbase = smem_addr(smem + LY::OFF_V + vs * LY::VBYTES);
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            // V block [BN keys][D] in 64-column boxes: MN-major B operand
-            const uint64_t bd = sdesc_sw128(vbase + kk * 16 * 128, BN * 128, 1024);
-            umma_ts(tmem + LY::TM_O + t * D, tmem + LY::TM_S + t * BN + kk * 8, bd, IDESC_O,
-                    (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(bar_pv(t));
-          if (t == 1) umma_commit(bar_vempty(vs));
-          if (j + 1 < nblk) {
-            // this tile's next scores go in behind its PV (issue order)
-            if (t == 0) {
-              if (!mbar_wait_spin(bar_kfull((j + 1) % KST), ((j + 1) / KST) & 1, abort_flag)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              k_next = true;
-            }
-            issue_qk(t, j + 1);
-            if (t == 1 && k_next) umma_commit(bar_kempty((j + 1) % KST));
-          }
-        }
-      }
-    }
-  } else {
-    // normalizer warpgroups: see prefill_pair_normalizer below
-    prefill_pair_normalizer<D, KST, VST>(A, smem, tmem, warp, lane, q0, bh0, kb0, nblk,
+  if (warp < 8) {
+    regs_inc<PAIR_REGS_NORM>();
+    // normalizer warpgroups: see prefill_pair_normalizer above
+    prefill_pair_normalizer<D, KST, VST, CAP>(A, smem, tmem, warp, lane, q0, bh0, kb0, nblk,
                                          bar_sfull(warp >> 2), bar_pfull(warp >> 2),
                                          bar_pv(warp >> 2), abort_flag);
+  
+  } else {
+    regs_dec<PAIR_REGS_CTRL>();
+    if (warp == 8) {
+      // ======================= TMA producer ===================================
+      if (lane == 0 && nblk > 0) {
+        tma_prefetch_desc(&tmq);
+        tma_prefetch_desc(&tmk);
+        tma_prefetch_desc(&tmv);
+        mbar_expect_tx(bar_q, 2 * LY::QBYTES);
+  #pragma unroll
+        for (int t = 0; t < 2; ++t)
+  #pragma unroll
+          for (int x = 0; x < D / 64; ++x)
+            tma_load_3d(smem_addr(smem + LY::OFF_Q + t * LY::QBYTES + x * TC_BM * 128), &tmq,
+                        bar_q, x * 64, q0, bh0 + t);
+        for (int j = 0; j < nblk; ++j) {
+          const int kb = kb0 + j;
+          const int ks = j % KST;
+          if (j >= KST && !mbar_wait(bar_kempty(ks), ((j / KST) + 1) & 1, abort_flag)) break;
+          mbar_expect_tx(bar_kfull(ks), LY::KBYTES);
+          uint8_t* kdst = smem + LY::OFF_K + ks * LY::KBYTES;
+  #pragma unroll
+          for (int x = 0; x < D / 64; ++x)
+            tma_load_3d(smem_addr(kdst + x * BN * 128), &tmk, bar_kfull(ks), x * 64, kb * BN,
+                        b * P.Hkv + g);
+          const int vs = j % VST;
+          if (j >= VST && !mbar_wait(bar_vempty(vs), ((j / VST) + 1) & 1, abort_flag)) break;
+          mbar_expect_tx(bar_vfull(vs), LY::VBYTES);
+          uint8_t* vdst = smem + LY::OFF_V + vs * LY::VBYTES;
+  #pragma unroll
+          for (int x = 0; x < D / 64; ++x)
+            tma_load_3d(smem_addr(vdst + x * BN * 128), &tmv, bar_vfull(vs), x * 64, kb * BN,
+                        b * P.Hkv + g);
+        }
+      }
+    } else if (warp == 9) {
+      // ======================= MMA issuer =====================================
+      if (lane == 0 && nblk > 0) {
+        constexpr uint32_t IDESC_S = idesc_bf16(TC_BM, BN, 0, 0);
+        constexpr uint32_t IDESC_O = idesc_bf16(TC_BM, D, 0, 1);
+        bool ok = mbar_wait_spin(bar_q, 0, abort_flag);
+        tc_fence_after();
+        auto issue_qk = [&](int t, int j) {
+          const uint32_t qbase = smem_addr(smem + LY::OFF_Q + t * LY::QBYTES);
+          const uint32_t kbase = smem_addr(smem + LY::OFF_K + (j % KST) * LY::KBYTES);
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad =
+                sdesc_sw128(qbase + (kk >> 2) * TC_BM * 128 + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(kbase + (kk >> 2) * BN * 128 + (kk & 3) * 32, 16, 1024);
+            umma_ss(tmem + LY::TM_S + t * BN, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar_sfull(t));
+        };
+        // prologue: both tiles' scores of the first block
+        if (ok && mbar_wait_spin(bar_kfull(0), 0, abort_flag)) {
+          tc_fence_after();
+          issue_qk(0, 0);
+          issue_qk(1, 0);
+          umma_commit(bar_kempty(0));
+        } else {
+          ok = false;
+        }
+        for (int j = 0; ok && j < nblk; ++j) {
+          const int vs = j % VST;
+          if (!mbar_wait_spin(bar_vfull(vs), (j / VST) & 1, abort_flag)) break;
+          bool k_next = false;
+          for (int t = 0; t < 2; ++t) {
+            if (!mbar_wait_spin(bar_pfull(t), j & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t vbase = smem_addr(smem + LY::OFF_V + vs * LY::VBYTES);
+  #pragma unroll
+            for (int kk = 0; kk < BN / 16; ++kk) {
+              // V block [BN keys][D] in 64-column boxes: MN-major B operand
+              const uint64_t bd = sdesc_sw128(vbase + kk * 16 * 128, BN * 128, 1024);
+              umma_ts(tmem + LY::TM_O + t * D, tmem + LY::TM_S + t * BN + kk * 8, bd, IDESC_O,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(bar_pv(t));
+            if (t == 1) umma_commit(bar_vempty(vs));
+            if (j + 1 < nblk) {
+              // this tile's next scores go in behind its PV (issue order)
+              if (t == 0) {
+                if (!mbar_wait_spin(bar_kfull((j + 1) % KST), ((j + 1) / KST) & 1, abort_flag)) {
+                  ok = false;
+                  break;
+                }
+                tc_fence_after();
+                k_next = true;
+              }
+              issue_qk(t, j + 1);
+              if (t == 1 && k_next) umma_commit(bar_kempty((j + 1) % KST));
+            }
+          }
+        }
+      }
+    }
   }
 
   tc_fence_before();

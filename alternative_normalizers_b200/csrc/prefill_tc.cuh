@@ -400,10 +400,11 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
     bool ovf = false;
     float lb = -INFINITY;  // lower bound of tau (threshold units)
     if constexpr (MODE == TC_ONLINE) {
-      // the softmax1 sink belongs to exactly one half of the row
-      const bool sink = P.norm == NATTN_SOFTMAX1 && half == 0;
-      m_run = sink ? 0.f : -INFINITY;
-      l_run = sink ? 1.f : 0.f;
+      // the sink (softmax1's logit 0, or a learned per-head logit, in log2
+      // units) belongs to exactly one half of the row
+      const float sink2 = (half == 0) ? sink_logit(P, h) * 1.4426950408889634f : -INFINITY;
+      m_run = sink2;
+      l_run = (sink2 == -INFINITY) ? 0.f : 1.f;
     } else {
       m_run = -INFINITY;
     }
@@ -476,15 +477,7 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
 #pragma unroll
         for (int c = 0; c < LDC / 64; ++c) {  // 64 scores -> 32 packed columns
           uint32_t pk[32];
-#pragma unroll
-          for (int k = 0; k < 64; k += 2) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(r[c * 64 + k]), fa, -msafe));
-            const float p1 =
-                fast_exp2(fmaf(__uint_as_float(r[c * 64 + k + 1]), fa, -msafe));
-            s0 += p0;
-            s1 += p1;
-            pk[k >> 1] = pack_bf16(p0, p1);
-          }
+          exp2_pack64(&r[c * 64], fa, msafe, s0, s1, pk);
           tmem_st32(paddr + c * 32, pk);
         }
         tmem_st_wait();

@@ -21,6 +21,9 @@ struct Problem {
   int causal;
   int window;
   float softcap;
+  // learned per-head attention sinks: logit of a value-0 sink in the
+  // softmax denominator of query head h (natural-log units), or null
+  const float* sinks;
   // paged mode (block_table != nullptr)
   const int32_t* block_table;
   const int32_t* seqlens;
@@ -52,6 +55,17 @@ __host__ __device__ __forceinline__ RowRange row_range(int Tq, int causal, int w
 
 __device__ __forceinline__ RowRange row_range(const Problem& P, int i, int L) {
   return row_range(P.Tq, P.causal, P.window, i, L);
+}
+
+// Logit of the value-0 sink in the denominator of query head h, natural-log
+// units: the learned per-head sink when given ("Attention variants",
+// TensorCAD, variants table, row "Attention sinks": a learned per-head term
+// in the softmax's denominator), 0 for softmax1 (its virtual logit-0 sink,
+// "HF Attention Normalizers", section "Important Limitations"), else -inf
+// (no sink).
+__device__ __forceinline__ float sink_logit(const Problem& P, int h) {
+  if (P.sinks != nullptr) return P.sinks[h];
+  return P.norm == NATTN_SOFTMAX1 ? 0.f : -INFINITY;
 }
 
 // Address of key (or value) row j of sequence b, kv head g.  Dense layout

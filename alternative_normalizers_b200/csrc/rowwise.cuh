@@ -238,7 +238,8 @@ __global__ void __launch_bounds__(ROW_THREADS)
       float mx = -INFINITY;
       for (int jj = tid; jj < n; jj += ROW_THREADS) mx = fmaxf(mx, sc[jj]);
       mx = block_max(mx, red);
-      if (P.norm == NATTN_SOFTMAX1) mx = fmaxf(mx, 0.f);
+      const float sink = sink_logit(P, h);  // -inf: no sink
+      mx = fmaxf(mx, sink);
       const float msafe = (mx == -INFINITY) ? 0.f : mx;
       float l = 0.f;
       for (int jj = tid; jj < n; jj += ROW_THREADS) {
@@ -247,7 +248,7 @@ __global__ void __launch_bounds__(ROW_THREADS)
         l += e;
       }
       l = block_sum(l, red);
-      if (P.norm == NATTN_SOFTMAX1) l += expf(-msafe);
+      if (sink != -INFINITY) l += expf(sink - msafe);
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       for (int jj = tid; jj < n; jj += ROW_THREADS) sc[jj] *= inv;
       stat = (l > 0.f) ? msafe + logf(l) : -INFINITY;

@@ -114,6 +114,20 @@ enum {
  *            visible key has a weight of exactly 0); softmax / softmax1: the
  *            number of visible keys.  0 for a row with no visible key.
  *
+ * Learned per-head attention sinks ("Attention variants: what to open up,
+ * and how far", TensorCAD, variants table, row "Attention sinks": a learned
+ * per-head term in the softmax's denominator; section "Recommendation":
+ * sinks as a parameter of the primitive):
+ *   sinks    float32 [Hq] or NULL, device memory, finite values (-inf: that
+ *            head has no sink).  With NATTN_SOFTMAX, query head h normalizes
+ *            over its visible scores plus one extra logit sinks[h] whose
+ *            value row is zero:
+ *                p_j = exp(z_j) / (exp(sinks[h]) + sum_k exp(z_k)),
+ *            row_stat = log(exp(sinks[h]) + sum_k exp(z_k)), and a row with
+ *            no visible key gets output 0 and row_stat sinks[h].  softmax1 is
+ *            the special case sinks[h] = 0.  Any other normalizer with sinks:
+ *            NATTN_EUNSUPPORTED.  4-byte aligned (NATTN_EALIGN).
+ *
  * window == 0 disables the sliding window; with causal it keeps keys with
  * 0 <= pos - j < window ("attention interface" wiki, section "common
  * flexattention patterns"); without causal it keeps |pos - j| < window.
@@ -141,6 +155,8 @@ typedef struct nattn_args {
   void* workspace;          /* device scratch, >= nattn_workspace_size(args) */
   size_t workspace_bytes;
   void* stream;             /* cudaStream_t */
+  const float* sinks;       /* learned per-head attention sinks, or NULL (see
+                               below); NATTN_SOFTMAX only                   */
 } nattn_args;
 
 /*
@@ -177,6 +193,60 @@ int nattn_fwd_ex(const nattn_args* a);
 /* Bytes of device scratch nattn_fwd_ex needs for these arguments (pointers
  * are not read).  Returns 0 for an invalid argument block. */
 size_t nattn_workspace_size(const nattn_args* a);
+
+/*
+ * Backward pass: gradients of L = sum(grad_out * O) with respect to q, k and
+ * v, recomputing the weights from the forward's saved row statistic ("HF
+ * Attention Normalizers", section "Important Limitations": softmax1 saves
+ * row max / denominator statistics and recomputes probabilities during the
+ * fused backward; the sparse kernels save one threshold per query row and
+ * recompute tiles during the fused backward).  Per row, the normalizer's
+ * Jacobian: softmax / softmax1 / sinks dz = p (g - sum p g); sparsemax
+ * dz = s (g - mean over the support of g), s = 1[p > 0]; 1.5-entmax
+ * dz = s (g - sum s g / sum s), s = sqrt(p); g = grad_out V^T.
+ *
+ * Dense mode only.  Layouts as in the forward:
+ *   q, k, v      bf16 [B,Hq,Tq,d], [B,Hkv,Tk,d], [B,Hkv,Tk,dv]: the forward's
+ *                inputs
+ *   out          bf16 [B,Hq,Tq,dv]: the forward's output
+ *   grad_out     bf16 [B,Hq,Tq,dv]: dL/dO
+ *   row_stat     float32 [B,Hq,Tq]: the forward's row_stat (log-sum-exp or
+ *                tau) for the same arguments
+ *   grad_q, grad_k, grad_v  bf16, shaped like q, k, v (outputs; grad_k and
+ *                grad_v sum over the query heads of each group)
+ * The mask, soft-cap, scale, normalizer and sinks must be the forward's.
+ * Supported: d == dv in {64, 128}; anything else NATTN_EUNSUPPORTED.  The
+ * caller passes scratch of nattn_bwd_workspace_size(a) bytes (one float per
+ * query row).  Asynchronous on `stream`; allocates nothing.  Returns NATTN_OK
+ * or a negative error code.
+ */
+typedef struct nattn_bwd_args {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* out;
+  const void* grad_out;
+  const float* row_stat;
+  void* grad_q;
+  void* grad_k;
+  void* grad_v;
+  int B, Hq, Hkv, Tq, Tk, d, dv;
+  float scale;
+  int normalizer;
+  int causal;
+  int window;
+  float softcap;
+  const float* sinks;       /* as in nattn_args (NATTN_SOFTMAX only)         */
+  void* workspace;
+  size_t workspace_bytes;
+  void* stream;             /* cudaStream_t */
+} nattn_bwd_args;
+
+int nattn_bwd(const nattn_bwd_args* a);
+
+/* Bytes of device scratch nattn_bwd needs (pointers are not read); 0 for an
+ * invalid or unsupported argument block. */
+size_t nattn_bwd_workspace_size(const nattn_bwd_args* a);
 
 /* Synchronises `stream`, returns the device status word of the current device
  * (NATTN_OK, NATTN_ETIMEOUT or NATTN_EBOUNDS; the first error recorded since

@@ -124,3 +124,38 @@ def test_short_form_paged_needs_device_allocations(L):
     rc = L.nattn_fwd(4096, 8192, 12288, 16384, None, 2, 8, 2, 1, 256, 128, 128,
                      0.088, 0, 1, 0, 0.0, 20480, 24576, None)
     assert rc == -1
+
+
+def test_sinks_only_with_softmax_and_aligned(L):
+    a = _args(L)
+    a.sinks = 4096
+    assert L.nattn_workspace_size(a) == 0          # softmax: valid, no scratch
+    for n in (1, 2, 3):                            # softmax1 / sparse: refused
+        a.normalizer = n
+        assert L.nattn_fwd_ex(a) == -2
+    a.normalizer = 0
+    a.sinks = 4098
+    assert L.nattn_fwd_ex(a) == -8
+
+
+def test_args_struct_layout_matches_c(tmp_path):
+    """The ctypes mirror of nattn_args has the C struct's size and field
+    offsets (checked with a small C program built against the header)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("needs gcc")
+    from alternative_normalizers_b200.binding import NattnArgs
+    names = [f[0] for f in NattnArgs._fields_]
+    src = tmp_path / "layout.c"
+    body = "".join(f'  printf("%zu\\n", offsetof(nattn_args, {n}));\n' for n in names)
+    src.write_text("#include <stddef.h>\n#include <stdio.h>\n#include \"nattn.h\"\n"
+                   "int main(void) {\n  printf(\"%zu\\n\", sizeof(nattn_args));\n"
+                   + body + "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src),
+                    "-o", str(exe)], check=True)
+    out = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True,
+                                          check=True).stdout.split()]
+    assert out[0] == ctypes.sizeof(NattnArgs)
+    assert out[1:] == [getattr(NattnArgs, n).offset for n in names]

@@ -169,12 +169,15 @@ def test_nattn_fwd_fullsize_paged(normalizer):
     import oracle
     from alternative_normalizers_b200.workloads import WORKLOADS, make_inputs
     w = WORKLOADS["paged_decode"]
+    import torch
     x = make_inputs(w)
-    assert x["block_table"].shape[1] == (w.len_range[1] + 63) // 64
+    # the short form's table stride is ceil(Tk / 64): pad the workload's table
+    stride = (w.len_range[1] + 63) // 64
+    table = torch.full((w.B, stride), -1, dtype=torch.int32)
+    table[:, :x["block_table"].shape[1]] = x["block_table"]
     rc, out, st = _call(x["q"].cuda(), x["k_pool"].cuda(), x["v_pool"].cuda(),
                         w.len_range[1], normalizer, True, scale=w.scale,
-                        block_table=x["block_table"].cuda(),
-                        seqlens=x["seqlens"].cuda())
+                        block_table=table.cuda(), seqlens=x["seqlens"].cuda())
     assert rc == 0
     lens = x["seqlens"].numpy()
     seqs = sorted({int(np.argmax(lens)), int(np.argmin(lens)), 5, 31})

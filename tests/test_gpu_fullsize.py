@@ -90,7 +90,8 @@ def support_check(w, x, rows, normalizer, tau_o, nnz_gpu):
         vis += ok.sum()
         sup_o += exact
         sup_g += g
-    assert banded <= max(2, len(rows) // 100)
+    # keys within the band of tau are rare: at most a few percent of rows
+    assert banded <= max(2, len(rows) // 20)
     return 1.0 - sup_g / vis, 1.0 - sup_o / vis
 
 
