@@ -58,53 +58,52 @@ constexpr int BWD_BQ = 64;        // queries per block (dK/dV kernel)
 
 enum BwdMode { BWD_DELTA = 0, BWD_DQ = 1 };
 
-// One score's contribution: from the raw dot product s, the row's saved
-// statistic, its delta and dP, the weight p (for dV) and dS (for dK, dQ).
-// sparse: 0 softmax family, 1 sparsemax, 2 1.5-entmax.  stat2 is the
-// log-sum-exp in log2 units (softmax family) or tau (sparse).
-struct BwdElem {
-  float scale, cap, zs2;  // zs2 = scale * log2(e)
-  float us;
-  int sparse;
-  __device__ __forceinline__ void eval(float s, float stat2, float delta, float dp, float& p,
+// One score's contribution, from the raw dot product s, the row's saved
+// statistic st (log-sum-exp in log2 units for the softmax family, tau for
+// the sparse normalizers), its delta and dP: the weight p (for dV) and dS
+// without the constant factor `scale` (applied to dQ and dK once, in the
+// epilogues; under the soft-cap dS keeps the 1 - tanh^2 of dz/ds).
+// KIND: 0 softmax / softmax1 / sinks, 1 sparsemax, 2 1.5-entmax.
+template <int KIND, bool CAP>
+struct BwdOp {
+  float a;  // CAP: scale / cap; else scale * log2(e) (KIND 0) or scale * us
+  float b;  // CAP: cap * log2(e) (KIND 0) or cap * us
+  __device__ __forceinline__ void eval(float s, float st, float dl, float dp, float& p,
                                        float& ds, float& w) const {
-    float dzds = scale, z;
-    if (cap > 0.f) {
-      const float t = fast_tanh(s * (scale / cap));
-      z = cap * t;
-      dzds = scale * (1.f - t * t);
+    float x, gcap = 1.f;
+    if (CAP) {
+      const float t = fast_tanh(s * a);
+      x = fmaf(t, b, -st);
+      gcap = fmaf(-t, t, 1.f);
     } else {
-      z = s * scale;
+      x = fmaf(s, a, -st);
     }
-    if (sparse == 0) {
-      p = fast_exp2(fmaf(z, 1.4426950408889634f, -stat2));
+    if (KIND == 0) {
+      p = fast_exp2(x);
       w = p;
+    } else if (KIND == 1) {
+      p = fmaxf(x, 0.f);
+      w = x > 0.f ? 1.f : 0.f;
     } else {
-      const float x = fmaf(z, us, -stat2);
       const float r = fmaxf(x, 0.f);
-      if (sparse == 1) {
-        p = r;
-        w = x > 0.f ? 1.f : 0.f;
-      } else {
-        p = r * r;
-        w = r;
-      }
+      p = r * r;
+      w = r;
     }
-    ds = w * (dp - delta) * dzds;
+    ds = w * (dp - dl);
+    if (CAP) ds *= gcap;
   }
 };
 
-__device__ __forceinline__ BwdElem make_elem(const BwdArgs& A) {
-  BwdElem e;
-  e.scale = A.P.scale;
-  e.cap = A.P.softcap;
-  e.zs2 = A.P.scale * 1.4426950408889634f;
-  e.us = A.us;
-  e.sparse = A.P.norm == NATTN_SPARSEMAX ? 1 : (A.P.norm == NATTN_ENTMAX15 ? 2 : 0);
-  return e;
+template <int KIND, bool CAP>
+__device__ __forceinline__ BwdOp<KIND, CAP> make_op(const BwdArgs& A) {
+  const float unit = (KIND == 0) ? 1.4426950408889634f : A.us;
+  BwdOp<KIND, CAP> op;
+  op.a = CAP ? A.P.scale / A.P.softcap : A.P.scale * unit;
+  op.b = CAP ? A.P.softcap * unit : 0.f;
+  return op;
 }
 
-// Saved statistic of a row in the units BwdElem::eval takes.
+// Saved statistic of a row in the units BwdOp::eval takes.
 __device__ __forceinline__ float bwd_stat2(const Problem& P, float st) {
   return (P.norm == NATTN_SOFTMAX || P.norm == NATTN_SOFTMAX1) ? st * 1.4426950408889634f
                                                                 : st;
@@ -145,7 +144,7 @@ __global__ void __launch_bounds__(256) bwd_delta_dot_kernel(BwdArgs A) {
 template <int D, int DV>
 struct BwdQLayout {
   static constexpr int BN = BWD_BN;
-  static constexpr int KST = 2, VST = 2;
+  static constexpr int KST = 4, VST = 4;  // K and V blocks in flight
   static constexpr int QBYTES = 128 * D * 2;
   static constexpr int OBYTES = 128 * DV * 2;
   static constexpr int KBYTES = BN * D * 2;
@@ -169,7 +168,7 @@ struct BwdQLayout {
   static_assert(ALLOC <= 227 * 1024, "shared memory budget");
 };
 
-template <int D, int DV, int MODE>
+template <int D, int DV, int MODE, int KIND, bool CAP>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmo,
                   const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
@@ -328,7 +327,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     if (!row_ok) rr = RowRange{1, 0};
     if (rr.hi > P.Tk - 1) rr.hi = P.Tk - 1;
     const size_t flat = (size_t)bh * P.Tq + qi;
-    const BwdElem E = make_elem(A);
+    const BwdOp<KIND, CAP> op = make_op<KIND, CAP>(A);
     const float stat2 = row_ok ? bwd_stat2(P, P.row_stat[flat]) : 0.f;
     const float dlt = (MODE == BWD_DQ && row_ok) ? A.delta[flat] : 0.f;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
@@ -348,17 +347,20 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       tmem_ld32(lane_base + LY::TM_DP + sb * BN + 32,
                 *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
       tmem_ld_wait();
+      // visible keys of this row relative to the block: [kl, kl + span]
       const int jb = (kb0 + j) * BN;
+      const int kl = rr.lo - jb;
+      const unsigned span = rr.hi >= rr.lo ? (unsigned)(rr.hi - rr.lo) : 0u;
+      const bool any = rr.hi >= rr.lo;
       uint32_t pk[32];
 #pragma unroll
       for (int k = 0; k < BN; k += 2) {
         float d2[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int kj = jb + k + e;
           float p, ds, w;
-          E.eval(__uint_as_float(s[k + e]), stat2, dlt, __uint_as_float(dp[k + e]), p, ds, w);
-          const bool vis = kj >= rr.lo && kj <= rr.hi;
+          op.eval(__uint_as_float(s[k + e]), stat2, dlt, __uint_as_float(dp[k + e]), p, ds, w);
+          const bool vis = any && (unsigned)(k + e - kl) <= span;
           d2[e] = vis ? ds : 0.f;
           if (MODE == BWD_DELTA && vis) {
             acc_wdp = fmaf(w, __uint_as_float(dp[k + e]), acc_wdp);
@@ -369,8 +371,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       }
       if (MODE == BWD_DQ) {
         // the dQ product of block j - 2 has read this dS buffer
-        if (j >= 2 &&
-            !__all_sync(0xffffffffu, mbar_wait(bar_dsempty(sb), ((j - 2) >> 1) & 1, abort_flag))) {
+        if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait_spin(bar_dsempty(sb), ((j - 2) >> 1) & 1,
+                                                              abort_flag))) {
           alive = false;
           break;
         }
@@ -399,13 +401,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           for (int k = 0; k < 32; ++k) r[k] = 0u;
         }
         if (row_ok) {
+          // dS left out the constant factor `scale`
+          const float sc = P.scale;
           uint4* dst = reinterpret_cast<uint4*>(drow + c * 32);
 #pragma unroll
           for (int k = 0; k < 32; k += 8)
-            dst[k / 8] = make_uint4(pack_bf16(__uint_as_float(r[k]), __uint_as_float(r[k + 1])),
-                                    pack_bf16(__uint_as_float(r[k + 2]), __uint_as_float(r[k + 3])),
-                                    pack_bf16(__uint_as_float(r[k + 4]), __uint_as_float(r[k + 5])),
-                                    pack_bf16(__uint_as_float(r[k + 6]), __uint_as_float(r[k + 7])));
+            dst[k / 8] = make_uint4(
+                pack_bf16(__uint_as_float(r[k]) * sc, __uint_as_float(r[k + 1]) * sc),
+                pack_bf16(__uint_as_float(r[k + 2]) * sc, __uint_as_float(r[k + 3]) * sc),
+                pack_bf16(__uint_as_float(r[k + 4]) * sc, __uint_as_float(r[k + 5]) * sc),
+                pack_bf16(__uint_as_float(r[k + 6]) * sc, __uint_as_float(r[k + 7]) * sc));
         }
       }
     }
@@ -423,6 +428,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 template <int D, int DV>
 struct BwdKVLayout {
   static constexpr int BQ = BWD_BQ;
+  static constexpr int QST = 3;  // query / dO / statistics slots in flight
   static constexpr int KBYTES = 128 * D * 2;
   static constexpr int VBYTES = 128 * DV * 2;
   static constexpr int QBYTES = BQ * D * 2;
@@ -430,14 +436,14 @@ struct BwdKVLayout {
   static constexpr int PBYTES = 128 * BQ * 2;  // one P^T or dS^T buffer [128 keys][64 q]
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KBYTES;
-  static constexpr int OFF_Q = OFF_V + VBYTES;        // 2 slots
-  static constexpr int OFF_O = OFF_Q + 2 * QBYTES;    // 2 slots
-  static constexpr int OFF_P = OFF_O + 2 * OBYTES;    // P^T, 2 buffers
-  static constexpr int OFF_DS = OFF_P + 2 * PBYTES;   // dS^T, 2 buffers
-  static constexpr int OFF_ST = OFF_DS + 2 * PBYTES;  // 2 slots of (stat2[64], delta[64])
-  static constexpr int OFF_BAR = OFF_ST + 2 * 2 * BQ * 4;
-  // kv, qfull[2], qempty[2], sfull[2], pfull[2], pempty[2], done
-  static constexpr int NBAR = 1 + 10 + 1;
+  static constexpr int OFF_Q = OFF_V + VBYTES;          // QST slots
+  static constexpr int OFF_O = OFF_Q + QST * QBYTES;    // QST slots
+  static constexpr int OFF_P = OFF_O + QST * OBYTES;    // P^T, 2 buffers
+  static constexpr int OFF_DS = OFF_P + 2 * PBYTES;     // dS^T, 2 buffers
+  static constexpr int OFF_ST = OFF_DS + 2 * PBYTES;    // QST slots of (stat2[64], delta[64])
+  static constexpr int OFF_BAR = OFF_ST + QST * 2 * BQ * 4;
+  // kv, qfull[QST], qempty[QST], sfull[2], pfull[2], pempty[2], done
+  static constexpr int NBAR = 1 + 2 * QST + 6 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int ALLOC = OFF_MISC + 16 + 1024;
   static constexpr int TM_S = 0;         // S^T buffer b at b * BQ
@@ -462,13 +468,13 @@ __device__ __forceinline__ RowRange key_query_range(const Problem& P, int j) {
   return RowRange{lo, hi};
 }
 
-template <int D, int DV>
+template <int D, int DV, int KIND, bool CAP>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmo,
                     const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                     BwdArgs A) {
   using LY = BwdKVLayout<D, DV>;
-  constexpr int BQ = LY::BQ;
+  constexpr int BQ = LY::BQ, QST = LY::QST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -493,20 +499,22 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + LY::OFF_BAR);
   const uint32_t bar_kv = smem_addr(&bars[0]);
   auto bar_qfull = [&](int s) { return smem_addr(&bars[1 + s]); };
-  auto bar_qempty = [&](int s) { return smem_addr(&bars[3 + s]); };
-  auto bar_sfull = [&](int s) { return smem_addr(&bars[5 + s]); };
-  auto bar_pfull = [&](int s) { return smem_addr(&bars[7 + s]); };
-  auto bar_pempty = [&](int s) { return smem_addr(&bars[9 + s]); };
-  const uint32_t bar_done = smem_addr(&bars[11]);
+  auto bar_qempty = [&](int s) { return smem_addr(&bars[1 + QST + s]); };
+  auto bar_sfull = [&](int s) { return smem_addr(&bars[1 + 2 * QST + s]); };
+  auto bar_pfull = [&](int s) { return smem_addr(&bars[3 + 2 * QST + s]); };
+  auto bar_pempty = [&](int s) { return smem_addr(&bars[5 + 2 * QST + s]); };
+  const uint32_t bar_done = smem_addr(&bars[7 + 2 * QST]);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + LY::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
-  float* stats = reinterpret_cast<float*>(smem + LY::OFF_ST);  // slot s: [s * 128, +128)
+  float* stats = reinterpret_cast<float*>(smem + LY::OFF_ST);  // slot q: [q * 128, +128)
 
   if (tid == 0) {
     mbar_init(bar_kv, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < QST; ++s) {
       mbar_init(bar_qfull(s), 1);
       mbar_init(bar_qempty(s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(bar_sfull(s), 1);
       mbar_init(bar_pfull(s), 4);
       mbar_init(bar_pempty(s), 1);
@@ -543,9 +551,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           tma_load_3d(smem_addr(smem + LY::OFF_V + x * 128 * 128), &tmv, bar_kv, x * 64, k0, bg);
       }
       for (int it = 0; it < nit; ++it) {
-        const int s = it & 1;
-        if (it >= 2 &&
-            !__all_sync(0xffffffffu, mbar_wait(bar_qempty(s), ((it - 2) >> 1) & 1, abort_flag)))
+        const int qs = it % QST;
+        if (it >= QST && !__all_sync(0xffffffffu, mbar_wait(bar_qempty(qs),
+                                                            ((it / QST) + 1) & 1, abort_flag)))
           break;
         int h, q0;
         item(it, h, q0);
@@ -553,18 +561,18 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         for (int c = lane; c < BQ; c += 32) {
           const int qi = q0 + c;
           const bool ok = qi < P.Tq;
-          stats[s * 2 * BQ + c] = ok ? bwd_stat2(P, P.row_stat[fbase + qi]) : 0.f;
-          stats[s * 2 * BQ + BQ + c] = ok ? A.delta[fbase + qi] : 0.f;
+          stats[qs * 2 * BQ + c] = ok ? bwd_stat2(P, P.row_stat[fbase + qi]) : 0.f;
+          stats[qs * 2 * BQ + BQ + c] = ok ? A.delta[fbase + qi] : 0.f;
         }
         __syncwarp();
         if (lane == 0) {
-          mbar_expect_tx(bar_qfull(s), LY::QBYTES + LY::OBYTES);
+          mbar_expect_tx(bar_qfull(qs), LY::QBYTES + LY::OBYTES);
           for (int x = 0; x < D / 64; ++x)
-            tma_load_3d(smem_addr(smem + LY::OFF_Q + s * LY::QBYTES + x * BQ * 128), &tmq,
-                        bar_qfull(s), x * 64, q0, b * P.Hq + h);
+            tma_load_3d(smem_addr(smem + LY::OFF_Q + qs * LY::QBYTES + x * BQ * 128), &tmq,
+                        bar_qfull(qs), x * 64, q0, b * P.Hq + h);
           for (int x = 0; x < DV / 64; ++x)
-            tma_load_3d(smem_addr(smem + LY::OFF_O + s * LY::OBYTES + x * BQ * 128), &tmo,
-                        bar_qfull(s), x * 64, q0, b * P.Hq + h);
+            tma_load_3d(smem_addr(smem + LY::OFF_O + qs * LY::OBYTES + x * BQ * 128), &tmo,
+                        bar_qfull(qs), x * 64, q0, b * P.Hq + h);
         }
         __syncwarp();
       }
@@ -581,13 +589,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       tc_fence_after();
       for (int it = 0; ok && it <= nit; ++it) {
         if (it < nit) {
-          const int s = it & 1;
-          if (!mbar_wait_spin(bar_qfull(s), (it >> 1) & 1, abort_flag)) break;
+          const int s = it & 1, qs = it % QST;
+          if (!mbar_wait_spin(bar_qfull(qs), (it / QST) & 1, abort_flag)) break;
           // TMEM buffer s last held item it - 2, read once pfull(it - 2)
           // completed, which the previous iteration waited for
           tc_fence_after();
-          const uint32_t qbase = smem_addr(smem + LY::OFF_Q + s * LY::QBYTES);
-          const uint32_t obase = smem_addr(smem + LY::OFF_O + s * LY::OBYTES);
+          const uint32_t qbase = smem_addr(smem + LY::OFF_Q + qs * LY::QBYTES);
+          const uint32_t obase = smem_addr(smem + LY::OFF_O + qs * LY::OBYTES);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             umma_ss(tmem + LY::TM_S + s * BQ,
@@ -603,13 +611,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           umma_commit(bar_sfull(s));
         }
         if (it >= 1) {
-          const int ip = it - 1, sp = ip & 1;
+          const int ip = it - 1, sp = ip & 1, qsp = ip % QST;
           if (!mbar_wait_spin(bar_pfull(sp), (ip >> 1) & 1, abort_flag)) break;
           tc_fence_after();
           const uint32_t pb = smem_addr(smem + LY::OFF_P + sp * LY::PBYTES);
           const uint32_t db = smem_addr(smem + LY::OFF_DS + sp * LY::PBYTES);
-          const uint32_t qbase = smem_addr(smem + LY::OFF_Q + sp * LY::QBYTES);
-          const uint32_t obase = smem_addr(smem + LY::OFF_O + sp * LY::OBYTES);
+          const uint32_t qbase = smem_addr(smem + LY::OFF_Q + qsp * LY::QBYTES);
+          const uint32_t obase = smem_addr(smem + LY::OFF_O + qsp * LY::OBYTES);
 #pragma unroll
           for (int kk = 0; kk < BQ / 16; ++kk) {
             // dV += P^T dO: A = P^T [128 keys][64 q] K-major, B = dO [64 q][DV] MN-major
@@ -621,7 +629,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                     sdesc_sw128(qbase + kk * 16 * 128, BQ * 128, 1024), IDESC_DK,
                     (ip > 0 || kk > 0) ? 1u : 0u);
           }
-          umma_commit(bar_qempty(sp));
+          umma_commit(bar_qempty(qsp));
           umma_commit(bar_pempty(sp));
         }
       }
@@ -634,16 +642,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const bool key_ok = kj < P.Tk;
     RowRange qr = key_query_range(P, kj);
     if (!key_ok) qr = RowRange{1, 0};
-    const BwdElem E = make_elem(A);
+    const BwdOp<KIND, CAP> op = make_op<KIND, CAP>(A);
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     bool alive = true;
     for (int it = 0; it < nit; ++it) {
-      const int s = it & 1;
+      const int s = it & 1, qs = it % QST;
       int h, q0;
       item(it, h, q0);
-      // qfull(s) carries the producer's stores of the rows' statistics (it
-      // has completed before sfull(s) can); sfull(s) the products
-      if (!__all_sync(0xffffffffu, mbar_wait_spin(bar_qfull(s), (it >> 1) & 1, abort_flag) &&
+      // qfull carries the producer's stores of the rows' statistics (it has
+      // completed before sfull(s) can); sfull(s) the products
+      if (!__all_sync(0xffffffffu, mbar_wait_spin(bar_qfull(qs), (it / QST) & 1, abort_flag) &&
                                        mbar_wait_spin(bar_sfull(s), (it >> 1) & 1, abort_flag))) {
         alive = false;
         break;
@@ -655,28 +663,36 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       tmem_ld32(lane_base + LY::TM_DP + s * BQ, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
       tmem_ld32(lane_base + LY::TM_DP + s * BQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
       tmem_ld_wait();
-      const float* st2 = stats + s * 2 * BQ;
-      const float* dl = st2 + BQ;
+      const float4* st4 = reinterpret_cast<const float4*>(stats + qs * 2 * BQ);
+      const float4* dl4 = st4 + BQ / 4;
+      // visible query columns of this key: [cl, cl + span]
+      const int cl = qr.lo - q0;
+      const unsigned span = qr.hi >= qr.lo ? (unsigned)(qr.hi - qr.lo) : 0u;
+      const bool any = qr.hi >= qr.lo;
       uint32_t ppk[32], dpk[32];
 #pragma unroll
-      for (int c = 0; c < BQ; c += 2) {
-        float pp[2], dd[2];
+      for (int c4 = 0; c4 < BQ; c4 += 4) {
+        const float4 sa = st4[c4 / 4], da = dl4[c4 / 4];
+        const float stv[4] = {sa.x, sa.y, sa.z, sa.w};
+        const float dlv[4] = {da.x, da.y, da.z, da.w};
+        float pp[4], dd[4];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int qi = q0 + c + e;
+        for (int e = 0; e < 4; ++e) {
           float p, ds, w;
-          E.eval(__uint_as_float(sv[c + e]), st2[c + e], dl[c + e], __uint_as_float(dp[c + e]),
-                 p, ds, w);
-          const bool vis = qi >= qr.lo && qi <= qr.hi;
+          op.eval(__uint_as_float(sv[c4 + e]), stv[e], dlv[e], __uint_as_float(dp[c4 + e]), p,
+                  ds, w);
+          const bool vis = any && (unsigned)(c4 + e - cl) <= span;
           pp[e] = vis ? p : 0.f;
           dd[e] = vis ? ds : 0.f;
         }
-        ppk[c >> 1] = pack_bf16(pp[0], pp[1]);
-        dpk[c >> 1] = pack_bf16(dd[0], dd[1]);
+        ppk[c4 >> 1] = pack_bf16(pp[0], pp[1]);
+        ppk[(c4 >> 1) + 1] = pack_bf16(pp[2], pp[3]);
+        dpk[c4 >> 1] = pack_bf16(dd[0], dd[1]);
+        dpk[(c4 >> 1) + 1] = pack_bf16(dd[2], dd[3]);
       }
       // the dK/dV products of item it - 2 have read these buffers
-      if (it >= 2 &&
-          !__all_sync(0xffffffffu, mbar_wait(bar_pempty(s), ((it - 2) >> 1) & 1, abort_flag))) {
+      if (it >= 2 && !__all_sync(0xffffffffu, mbar_wait_spin(bar_pempty(s), ((it - 2) >> 1) & 1,
+                                                              abort_flag))) {
         alive = false;
         break;
       }
@@ -690,7 +706,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const bool have =
         __all_sync(0xffffffffu, alive && nit > 0 && mbar_wait(bar_done, 0, abort_flag));
     tc_fence_after();
-    auto store = [&](uint32_t tcol, bf16* dst, int cols) {
+    // dS left out the constant factor `scale`: dK takes it here
+    auto store = [&](uint32_t tcol, bf16* dst, int cols, float sc) {
 #pragma unroll 1
       for (int c = 0; c < cols / 32; ++c) {
         uint32_t r[32];
@@ -705,16 +722,17 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           uint4* o = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
           for (int k = 0; k < 32; k += 8)
-            o[k / 8] = make_uint4(pack_bf16(__uint_as_float(r[k]), __uint_as_float(r[k + 1])),
-                                  pack_bf16(__uint_as_float(r[k + 2]), __uint_as_float(r[k + 3])),
-                                  pack_bf16(__uint_as_float(r[k + 4]), __uint_as_float(r[k + 5])),
-                                  pack_bf16(__uint_as_float(r[k + 6]), __uint_as_float(r[k + 7])));
+            o[k / 8] = make_uint4(
+                pack_bf16(__uint_as_float(r[k]) * sc, __uint_as_float(r[k + 1]) * sc),
+                pack_bf16(__uint_as_float(r[k + 2]) * sc, __uint_as_float(r[k + 3]) * sc),
+                pack_bf16(__uint_as_float(r[k + 4]) * sc, __uint_as_float(r[k + 5]) * sc),
+                pack_bf16(__uint_as_float(r[k + 6]) * sc, __uint_as_float(r[k + 7]) * sc));
         }
       }
     };
     const size_t krow = ((size_t)b * P.Hkv + g) * P.Tk + kj;
-    store(LY::TM_DK, A.dk + krow * D, D);
-    store(LY::TM_DV, A.dv + krow * DV, DV);
+    store(LY::TM_DK, A.dk + krow * D, D, P.scale);
+    store(LY::TM_DV, A.dv + krow * DV, DV, 1.f);
   }
 
   tc_fence_before();

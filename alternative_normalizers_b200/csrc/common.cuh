@@ -57,16 +57,37 @@ __device__ __forceinline__ float fast_exp2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// Packed pairs of fp32 (sm_100 f32x2 arithmetic: one instruction does the
+// operation on both halves of a 64-bit register pair).
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0,
+                                      float b1, float c0, float c1) {
+  asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0,
+                                      float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // p_k = 2^(r_k * fa - m) for 64 scores held as raw bits; returns the bf16
 // pairs packed for a TMEM store and adds the fp32 weights into s0 / s1.
+// Pairs of scores share one f32x2 FFMA and one f32x2 add.
 __device__ __forceinline__ void exp2_pack64(const uint32_t* r, float fa, float m, float& s0,
                                             float& s1, uint32_t (&pk)[32]) {
 #pragma unroll
   for (int k = 0; k < 64; k += 2) {
-    const float p0 = fast_exp2(fmaf(__uint_as_float(r[k]), fa, -m));
-    const float p1 = fast_exp2(fmaf(__uint_as_float(r[k + 1]), fa, -m));
-    s0 += p0;
-    s1 += p1;
+    float x0, x1;
+    ffma2(x0, x1, __uint_as_float(r[k]), __uint_as_float(r[k + 1]), fa, fa, -m, -m);
+    const float p0 = fast_exp2(x0);
+    const float p1 = fast_exp2(x1);
+    fadd2(s0, s1, s0, s1, p0, p1);
     pk[k >> 1] = pack_bf16(p0, p1);
   }
 }

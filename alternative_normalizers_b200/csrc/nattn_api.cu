@@ -611,6 +611,50 @@ size_t bwd_workspace(const nattn_bwd_args* a) {
   return up256((size_t)a->B * a->Hq * a->Tq * 4);
 }
 
+// One backward: the per-row delta (a dot product for the softmax family,
+// the dQ kernel's DELTA mode for the sparse normalizers), then the dQ kernel,
+// then the dK/dV kernel; KIND 0 softmax family, 1 sparsemax, 2 1.5-entmax.
+template <int D, int KIND, bool CAP>
+int launch_bwd_kind(const nattn_bwd_args* a, BwdArgs& A, cudaStream_t st) {
+  const long long BHq = (long long)a->B * a->Hq, BHkv = (long long)a->B * a->Hkv;
+  // dQ kernel: 128-row query tiles, 64-key blocks
+  CUtensorMap mq, mo, mk, mv;
+  if (!make_map_3d(&mq, a->q, D, a->Tq, BHq, 128) ||
+      !make_map_3d(&mo, a->grad_out, D, a->Tq, BHq, 128) ||
+      !make_map_3d(&mk, a->k, D, a->Tk, BHkv, BWD_BN) ||
+      !make_map_3d(&mv, a->v, D, a->Tk, BHkv, BWD_BN))
+    return NATTN_ECUDA;
+  const unsigned gq = (unsigned)(BHq * ((a->Tq + 127) / 128));
+  using LQ = BwdQLayout<D, D>;
+  if constexpr (KIND != 0) {
+    auto k = bwd_dq_kernel<D, D, BWD_DELTA, KIND, CAP>;
+    if (allow_smem(k, LQ::ALLOC) != cudaSuccess) return NATTN_ECUDA;
+    k<<<gq, BWD_THREADS, LQ::ALLOC, st>>>(mq, mo, mk, mv, A);
+  } else {
+    const size_t rows = (size_t)BHq * a->Tq;
+    bwd_delta_dot_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(A);
+  }
+  if (check_launch() != NATTN_OK) return NATTN_ECUDA;
+  {
+    auto k = bwd_dq_kernel<D, D, BWD_DQ, KIND, CAP>;
+    if (allow_smem(k, LQ::ALLOC) != cudaSuccess) return NATTN_ECUDA;
+    k<<<gq, BWD_THREADS, LQ::ALLOC, st>>>(mq, mo, mk, mv, A);
+    if (check_launch() != NATTN_OK) return NATTN_ECUDA;
+  }
+  // dK/dV kernel: 128-key tiles, 64-row query blocks
+  if (!make_map_3d(&mq, a->q, D, a->Tq, BHq, BWD_BQ) ||
+      !make_map_3d(&mo, a->grad_out, D, a->Tq, BHq, BWD_BQ) ||
+      !make_map_3d(&mk, a->k, D, a->Tk, BHkv, 128) ||
+      !make_map_3d(&mv, a->v, D, a->Tk, BHkv, 128))
+    return NATTN_ECUDA;
+  using LK = BwdKVLayout<D, D>;
+  auto k = bwd_dkdv_kernel<D, D, KIND, CAP>;
+  if (allow_smem(k, LK::ALLOC) != cudaSuccess) return NATTN_ECUDA;
+  const unsigned gk = (unsigned)(BHkv * ((a->Tk + 127) / 128));
+  k<<<gk, BWD_THREADS, LK::ALLOC, st>>>(mq, mo, mk, mv, A);
+  return check_launch();
+}
+
 template <int D>
 int launch_bwd(const nattn_bwd_args* a, cudaStream_t st) {
   BwdArgs A;
@@ -640,44 +684,15 @@ int launch_bwd(const nattn_bwd_args* a, cudaStream_t st) {
   A.dv = static_cast<bf16*>(a->grad_v);
   A.delta = static_cast<float*>(a->workspace);
   A.us = (a->normalizer == NATTN_ENTMAX15) ? 0.5f : 1.0f;
-  const bool sparse = a->normalizer == NATTN_SPARSEMAX || a->normalizer == NATTN_ENTMAX15;
-  const long long BHq = (long long)a->B * a->Hq, BHkv = (long long)a->B * a->Hkv;
-  // dQ kernel: 128-row query tiles, 64-key blocks
-  CUtensorMap mq, mo, mk, mv;
-  if (!make_map_3d(&mq, a->q, D, a->Tq, BHq, 128) ||
-      !make_map_3d(&mo, a->grad_out, D, a->Tq, BHq, 128) ||
-      !make_map_3d(&mk, a->k, D, a->Tk, BHkv, BWD_BN) ||
-      !make_map_3d(&mv, a->v, D, a->Tk, BHkv, BWD_BN))
-    return NATTN_ECUDA;
-  const unsigned gq = (unsigned)(BHq * ((a->Tq + 127) / 128));
-  using LQ = BwdQLayout<D, D>;
-  if (sparse) {
-    auto k = bwd_dq_kernel<D, D, BWD_DELTA>;
-    if (allow_smem(k, LQ::ALLOC) != cudaSuccess) return NATTN_ECUDA;
-    k<<<gq, BWD_THREADS, LQ::ALLOC, st>>>(mq, mo, mk, mv, A);
-  } else {
-    const size_t rows = (size_t)BHq * a->Tq;
-    bwd_delta_dot_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(A);
+  const bool cap = a->softcap > 0.f;
+  switch (a->normalizer) {
+    case NATTN_SPARSEMAX:
+      return cap ? launch_bwd_kind<D, 1, true>(a, A, st) : launch_bwd_kind<D, 1, false>(a, A, st);
+    case NATTN_ENTMAX15:
+      return cap ? launch_bwd_kind<D, 2, true>(a, A, st) : launch_bwd_kind<D, 2, false>(a, A, st);
+    default:
+      return cap ? launch_bwd_kind<D, 0, true>(a, A, st) : launch_bwd_kind<D, 0, false>(a, A, st);
   }
-  if (check_launch() != NATTN_OK) return NATTN_ECUDA;
-  {
-    auto k = bwd_dq_kernel<D, D, BWD_DQ>;
-    if (allow_smem(k, LQ::ALLOC) != cudaSuccess) return NATTN_ECUDA;
-    k<<<gq, BWD_THREADS, LQ::ALLOC, st>>>(mq, mo, mk, mv, A);
-    if (check_launch() != NATTN_OK) return NATTN_ECUDA;
-  }
-  // dK/dV kernel: 128-key tiles, 64-row query blocks
-  if (!make_map_3d(&mq, a->q, D, a->Tq, BHq, BWD_BQ) ||
-      !make_map_3d(&mo, a->grad_out, D, a->Tq, BHq, BWD_BQ) ||
-      !make_map_3d(&mk, a->k, D, a->Tk, BHkv, 128) ||
-      !make_map_3d(&mv, a->v, D, a->Tk, BHkv, 128))
-    return NATTN_ECUDA;
-  using LK = BwdKVLayout<D, D>;
-  auto k = bwd_dkdv_kernel<D, D>;
-  if (allow_smem(k, LK::ALLOC) != cudaSuccess) return NATTN_ECUDA;
-  const unsigned gk = (unsigned)(BHkv * ((a->Tk + 127) / 128));
-  k<<<gk, BWD_THREADS, LK::ALLOC, st>>>(mq, mo, mk, mv, A);
-  return check_launch();
 }
 
 int run_bwd(const nattn_bwd_args* a) {

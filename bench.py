@@ -571,6 +571,48 @@ def sparse_decode_bytes(r, n):
             "total": kb + vb + sb + qo, "v_pages": vpages}
 
 
+class BwdRunner:
+    """The backward pass of one dense workload: the forward runs once to give
+    the saved output and row statistic, then every timed call is one
+    nattn_bwd (delta pass, dQ kernel, dK/dV kernel).  Useful FLOPs are 2.5x
+    the forward's (five products of the forward's size against two)."""
+
+    def __init__(self, w, dev):
+        import torch
+        from alternative_normalizers_b200 import binding
+        from alternative_normalizers_b200.workloads import make_inputs
+        self.w, self.binding = w, binding
+        x = make_inputs(w)
+        g = torch.Generator().manual_seed(w.seed + 500)
+        dout = torch.randn(w.B, w.Hq, w.Tq, w.dv, generator=g).to(torch.bfloat16)
+        self.x = {k: v.to(dev) for k, v in x.items()}
+        self.dout = dout.to(dev)
+        self.args, self.keep = {}, []
+        for n in w.normalizers:
+            out, st, _ = binding.attention(self.x["q"], self.x["k"], self.x["v"],
+                                           normalizer=n, causal=w.causal,
+                                           window=w.window, softcap=w.softcap,
+                                           scale=w.scale)
+            dq, dk, dv = (torch.empty_like(self.x[t]) for t in ("q", "k", "v"))
+            a = binding.build_bwd_args(self.x["q"], self.x["k"], self.x["v"], out, st,
+                                       self.dout, dq, dk, dv, normalizer=n,
+                                       causal=w.causal, window=w.window,
+                                       softcap=w.softcap, scale=w.scale)
+            ws = torch.empty(binding.nattn_bwd_workspace_size(a), dtype=torch.uint8,
+                             device=dev)
+            a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+            self.keep += [out, st, dq, dk, dv, ws]
+            self.args[n] = a
+
+    def call(self, n):
+        rc = self.binding.nattn_bwd(self.args[n])
+        if rc != 0:
+            raise RuntimeError(f"nattn_bwd({n}) failed: {rc}")
+
+    def units(self):
+        return 2.5 * self.w.useful_flops()
+
+
 def detail(args, dev, flush):
     """The other workload shapes, each normalizer timed like the headline."""
     import torch
@@ -618,6 +660,43 @@ def detail(args, dev, flush):
             torch.cuda.empty_cache()
         except Exception as exc:  # report, keep the headline line
             res[name] = {"error": repr(exc)[:200]}
+    peaks = load_peaks()[0]
+    # backward pass (fused, recomputing the weights from the saved statistic)
+    for name in ("qwen3_8b_prefill", "sparse_prefill_t1"):
+        w = WORKLOADS[name]
+        try:
+            r = BwdRunner(w, dev)
+            per = time_runner(r, max(3, args.steps // 2), 2, flush)
+            u = r.units()
+            vals = {n: round(u / (t * 1e-3) / 1e12, 1) for n, t in per.items()}
+            res[name + "_backward"] = {
+                "unit": "useful TFLOP/s (2.5x the forward's useful FLOPs)",
+                "value": vals, "ms": {n: round(t, 4) for n, t in per.items()},
+                "roofline_frac": {n: round(v / peaks["bf16_tflops"], 4)
+                                  for n, v in vals.items()},
+                "roofline_denominator": "of measured bf16_tflops (burst)"}
+            del r
+            torch.cuda.empty_cache()
+        except Exception as exc:
+            res[name + "_backward"] = {"error": repr(exc)[:200]}
+    # learned per-head sinks on the headline shape (softmax with sinks[h])
+    try:
+        w = replace(WORKLOADS["qwen3_8b_prefill"], normalizers=("softmax",))
+        r = Runner(w, dev)
+        g = torch.Generator().manual_seed(77)
+        sinks = (torch.randn(w.Hq, generator=g) * 2).to(dev)
+        r.args["softmax"].sinks = sinks.data_ptr()
+        per = time_runner(r, max(3, args.steps // 2), 2, flush)
+        v = r.units() / (per["softmax"] * 1e-3) / 1e12
+        res["qwen3_8b_prefill_sinks"] = {
+            "unit": "useful TFLOP/s", "value": {"softmax+sinks": round(v, 1)},
+            "ms": {"softmax+sinks": round(per["softmax"], 4)},
+            "roofline_frac": {"softmax+sinks": round(v / peaks["bf16_tflops"], 4)},
+            "roofline_denominator": "of measured bf16_tflops (burst)"}
+        del r, sinks
+        torch.cuda.empty_cache()
+    except Exception as exc:
+        res["qwen3_8b_prefill_sinks"] = {"error": repr(exc)[:200]}
     return res
 
 

@@ -110,3 +110,88 @@ def test_backward_unsupported_head_dim():
     st = torch.zeros(1, 2, 16, device="cuda")
     with pytest.raises(NattnError):
         attention_backward(x, x, x, x, st, x, normalizer="softmax")
+
+
+def _rows_grad(x, w, dout, normalizer, b, h, rows):
+    """Oracle dZ rows (and weights) of query head h, composed from the
+    oracle's row functions: p from the forward row normalizer, dz from its
+    Jacobian; returns {i: (visible key indices, p, dS = dz * scale)}."""
+    import oracle
+    q = oracle.attention._f64(x["q"][b, h])
+    g = h // (w.Hq // w.Hkv)
+    k = oracle.attention._f64(x["k"][b, g])
+    v = oracle.attention._f64(x["v"][b, g])
+    do = oracle.attention._f64(dout[b, h])
+    ok_all = oracle.allowed_matrix(w.Tq, w.Tk, w.causal, w.window)
+    res = {}
+    for i in rows:
+        idx = np.nonzero(ok_all[i])[0]
+        z = oracle.transform_scores(q[i] @ k[idx].T, w.scale, w.softcap)
+        p, _ = oracle.normalize_row(z, normalizer)
+        dz = oracle.row_vjp(p, do[i] @ v[idx].T, normalizer)
+        res[i] = (idx, p, dz * w.scale)
+    return res, q, k, do
+
+
+@pytest.mark.parametrize("name,normalizer", [("qwen3_8b_prefill", "softmax"),
+                                             ("sparse_prefill_t1", "sparsemax"),
+                                             ("sparse_prefill_t1", "entmax15")])
+def test_backward_fullsize(name, normalizer):
+    """Full workload size, in the launch configuration the benchmark times:
+    dQ on sampled rows, dK / dV on the last key tile of one key/value head
+    (seen, under the causal mask, only by the last 128 query rows of each
+    head of its group), and for softmax the column-sum identities
+    sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i that hold at any size."""
+    import torch
+    import oracle
+    from alternative_normalizers_b200 import attention, attention_backward
+    from alternative_normalizers_b200.workloads import WORKLOADS, make_inputs
+    from tests._util import fullsize_rows
+    w = WORKLOADS[name]
+    x = make_inputs(w)
+    gen = torch.Generator().manual_seed(w.seed + 500)
+    dout = torch.randn(w.B, w.Hq, w.Tq, w.dv, generator=gen).to(torch.bfloat16)
+    qc, kc, vc = x["q"].cuda(), x["k"].cuda(), x["v"].cuda()
+    out, st, _ = attention(qc, kc, vc, normalizer=normalizer, causal=w.causal,
+                           scale=w.scale)
+    dq, dk, dv = attention_backward(qc, kc, vc, out, st, dout.cuda(),
+                                    normalizer=normalizer, causal=w.causal,
+                                    scale=w.scale)
+    torch.cuda.synchronize()
+    dq, dk, dv = (t.float().cpu().numpy() for t in (dq, dk, dv))
+    assert np.isfinite(dq).all() and np.isfinite(dk).all() and np.isfinite(dv).all()
+    # dQ rows
+    rows = fullsize_rows(w, 512)
+    got, want = [], []
+    for (b, h) in sorted({(int(r[0]), int(r[1])) for r in rows}):
+        sel = [int(r[2]) for r in rows if r[0] == b and r[1] == h]
+        res, q, k, _ = _rows_grad(x, w, dout, normalizer, b, h, sel)
+        for i in sel:
+            idx, _, ds = res[i]
+            want.append(ds @ k[idx])
+            got.append(dq[b, h, i])
+    check_grad(np.array(got), np.array(want), f"dq rows {name}/{normalizer}")
+    # dK, dV of the last key tile of kv head 0 of batch 0
+    b, g = 0, 0
+    j0 = w.Tk - 128
+    group = w.Hq // w.Hkv
+    rk = np.zeros((128, w.d))
+    rv = np.zeros((128, w.dv))
+    for h in range(g * group, (g + 1) * group):
+        sel = list(range(j0 - (w.Tk - w.Tq), w.Tq))
+        res, q, _, do = _rows_grad(x, w, dout, normalizer, b, h, sel)
+        for i in sel:
+            idx, p, ds = res[i]
+            m = idx >= j0
+            rk[idx[m] - j0] += ds[m, None] * q[i][None, :]
+            rv[idx[m] - j0] += p[m, None] * do[i][None, :]
+    check_grad(dk[b, g, j0:], rk, f"dk last tile {name}/{normalizer}")
+    check_grad(dv[b, g, j0:], rv, f"dv last tile {name}/{normalizer}")
+    if normalizer == "softmax":
+        for b in range(w.B):
+            for g in range(w.Hkv):
+                s_k = dk[b, g].sum(0)
+                assert np.abs(s_k).max() <= 2 ** -7 * np.abs(dk[b, g]).sum(0).max() + 1e-3
+                s_v = dv[b, g].sum(0)
+                want_v = dout[b, g * group:(g + 1) * group].float().numpy().sum((0, 1))
+                assert np.abs(s_v - want_v).max() <= 2 ** -7 * np.abs(dv[b, g]).sum(0).max() + 1e-3
