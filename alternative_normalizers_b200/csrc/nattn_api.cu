@@ -112,6 +112,15 @@ size_t bytes_to_alloc_end(const void* p) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Streaming multiprocessors of the current device.
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+    return 148;
+  return n;
+}
+
 // Per-device one-time kernel attribute set-up (dynamic shared memory opt-in).
 template <class K>
 cudaError_t allow_smem(K kernel, int bytes) {
@@ -337,7 +346,10 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
         auto kp = cap ? prefill_pair_kernel<D, KST, VST, true>
                       : prefill_pair_kernel<D, KST, VST, false>;
         if (allow_smem(kp, PL::ALLOC) != cudaSuccess) return NATTN_ECUDA;
-        const unsigned pgrid = (unsigned)((long long)a->B * (a->Hq / 2) * ntq);
+        // persistent: one CTA per SM (shared memory and TMEM allow one), each
+        // walking its share of the tiles
+        const long long ntiles = (long long)a->B * (a->Hq / 2) * ntq;
+        const unsigned pgrid = (unsigned)(ntiles < num_sms() ? ntiles : num_sms());
         kp<<<pgrid, PAIR_THREADS, PL::ALLOC, st>>>(mq, mk, mv, A);
         return check_launch();
       }

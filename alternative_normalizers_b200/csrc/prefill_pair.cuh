@@ -47,8 +47,8 @@ struct PairLayout {
   static constexpr int OFF_K = 2 * QBYTES;
   static constexpr int OFF_V = OFF_K + KST * KBYTES;
   static constexpr int OFF_BAR = OFF_V + VST * VBYTES;
-  // q, kfull/kempty, vfull/vempty, sfull[2], pfull[2], pvdone[2]
-  static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 6;
+  // q, kfull/kempty, vfull/vempty, sfull[2], pfull[2], pvdone[2], qempty
+  static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 6 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;
@@ -59,13 +59,53 @@ struct PairLayout {
   static_assert(ALLOC <= 227 * 1024, "shared memory budget");
 };
 
+// One unit of work: the same 128 query rows of the two query heads h0, h0 + 1
+// (one GQA group) of batch b, and the visible key blocks [kb0, kb0 + nblk).
+struct PairTile {
+  int b, h0, g, bh0, q0, kb0, nblk;
+};
+
+// Tile of heaviest-first rank `rank`: under the causal mask the last query
+// tiles see the most keys, so ranks walk the query tiles from the last.
+__device__ __forceinline__ PairTile pair_tile(const Problem& P, int rank) {
+  const int ntq = (P.Tq + TC_BM - 1) / TC_BM;
+  const int HP = P.Hq / 2;  // head pairs per batch
+  const int BP = P.B * HP;
+  const int qt = P.causal ? (ntq - 1 - rank / BP) : (rank / BP);
+  const int bp = rank % BP;
+  PairTile T;
+  T.b = bp / HP;
+  T.h0 = 2 * (bp % HP);
+  T.g = T.h0 / (P.Hq / P.Hkv);
+  T.bh0 = T.b * P.Hq + T.h0;
+  T.q0 = qt * TC_BM;
+  const int qlast = min(T.q0 + TC_BM - 1, P.Tq - 1);
+  const RowRange r_first = row_range(P, T.q0, P.Tk);
+  const RowRange r_last = row_range(P, qlast, P.Tk);
+  const int klo = max(0, r_first.lo);
+  const int khi = min(P.Tk - 1, r_last.hi);
+  T.kb0 = klo / 128;
+  T.nblk = (khi >= klo) ? (khi / 128 - T.kb0 + 1) : 0;
+  return T;
+}
+
+// Persistent schedule: CTA c of G takes, in round k, rank k*G + c (k even)
+// or k*G + G-1-c (k odd).  Over heaviest-first ranks this snake evens out
+// the CTAs' total work.  Ranks only grow, so the first one past the end
+// ends the CTA's walk.
+__device__ __forceinline__ int pair_rank(int round, int c, int G) {
+  return round * G + ((round & 1) ? (G - 1 - c) : c);
+}
+
 // One normalizer warp of tile t = warp / 4: thread = query row = TMEM lane of
 // its lane quarter.  The S row is read from TMEM once per block and held in
 // registers (128 values) for the maximum and the exponentials.
+// `g0` counts the blocks of the CTA's earlier tiles: barrier phases run on
+// across tiles.  Returns false if a wait gave up.
 template <int D, int KST, int VST, bool CAP>
-__device__ __forceinline__ void prefill_pair_normalizer(
+__device__ __forceinline__ bool prefill_pair_normalizer(
     const TcArgs& A, uint8_t* smem, uint32_t tmem, int warp, int lane, int q0, int bh0,
-    int kb0, int nblk, uint32_t bar_sf, uint32_t bar_pf, uint32_t bar_pvt,
+    int kb0, int nblk, int g0, uint32_t bar_sf, uint32_t bar_pf, uint32_t bar_pvt,
     volatile int* abort_flag) {
   using LY = PairLayout<D, KST, VST>;
   constexpr int BN = LY::BN;
@@ -93,7 +133,7 @@ __device__ __forceinline__ void prefill_pair_normalizer(
   bool alive = true;
 
   for (int j = 0; j < nblk; ++j) {
-    if (!__all_sync(0xffffffffu, mbar_wait_spin(bar_sf, j & 1, abort_flag))) {
+    if (!__all_sync(0xffffffffu, mbar_wait_spin(bar_sf, (g0 + j) & 1, abort_flag))) {
       alive = false;
       break;
     }
@@ -142,7 +182,7 @@ __device__ __forceinline__ void prefill_pair_normalizer(
     tmem_st_wait();
     l_run = l_run * alpha + (s0 + s1);
     if (__any_sync(0xffffffffu, resc) && j > 0) {
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_pvt, (j - 1) & 1, abort_flag))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_pvt, (g0 + j - 1) & 1, abort_flag))) {
         alive = false;
         break;
       }
@@ -166,7 +206,7 @@ __device__ __forceinline__ void prefill_pair_normalizer(
 
   // ---- epilogue -------------------------------------------------------------
   const bool have_o = __all_sync(
-      0xffffffffu, alive && nblk > 0 && mbar_wait(bar_pvt, (nblk - 1) & 1, abort_flag));
+      0xffffffffu, alive && nblk > 0 && mbar_wait(bar_pvt, (g0 + nblk - 1) & 1, abort_flag));
   tc_fence_after();
   const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
   const float msafe = (m_run == -INFINITY) ? 0.f : m_run;
@@ -197,6 +237,7 @@ __device__ __forceinline__ void prefill_pair_normalizer(
   }
   if (row_ok && P.row_stat) P.row_stat[flat] = stat;
   if (row_ok && P.row_nnz) P.row_nnz[flat] = rr.hi >= rr.lo ? rr.hi - rr.lo + 1 : 0;
+  return alive;
 }
 
 template <int D, int KST, int VST, bool CAP>
@@ -212,25 +253,10 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
   const Problem& P = A.P;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // ---- tile selection: (query tile, batch, pair of heads of one group) ---
+  // ---- persistent: this CTA walks tiles pair_rank(0..), see pair_rank ----
   const int ntq = (P.Tq + TC_BM - 1) / TC_BM;
-  const int HP = P.Hq / 2;                 // head pairs per batch
-  const int BP = P.B * HP;
-  const int rank = blockIdx.x;
-  const int qt = P.causal ? (ntq - 1 - rank / BP) : (rank / BP);
-  const int bp = rank % BP;
-  const int b = bp / HP;
-  const int h0 = 2 * (bp % HP);
-  const int g = h0 / (P.Hq / P.Hkv);
-  const int bh0 = b * P.Hq + h0;           // tile t reads query head h0 + t
-  const int q0 = qt * TC_BM;
-  const int qlast = min(q0 + TC_BM - 1, P.Tq - 1);
-  const RowRange r_first = row_range(P, q0, P.Tk);
-  const RowRange r_last = row_range(P, qlast, P.Tk);
-  const int klo = max(0, r_first.lo);
-  const int khi = min(P.Tk - 1, r_last.hi);
-  const int kb0 = klo / BN;
-  const int nblk = (khi >= klo) ? (khi / BN - kb0 + 1) : 0;
+  const int ntiles = P.B * (P.Hq / 2) * ntq;
+  const int G = gridDim.x, cta = blockIdx.x;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + LY::OFF_BAR);
   const uint32_t bar_q = smem_addr(&bars[0]);
@@ -241,6 +267,8 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
   auto bar_sfull = [&](int t) { return smem_addr(&bars[1 + 2 * KST + 2 * VST + t]); };
   auto bar_pfull = [&](int t) { return smem_addr(&bars[1 + 2 * KST + 2 * VST + 2 + t]); };
   auto bar_pv = [&](int t) { return smem_addr(&bars[1 + 2 * KST + 2 * VST + 4 + t]); };
+  // the MMAs that read the Q tiles of a tile are done: the next tile's Q may load
+  const uint32_t bar_qempty = smem_addr(&bars[1 + 2 * KST + 2 * VST + 6]);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + LY::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
 
@@ -259,6 +287,7 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
       mbar_init(bar_pfull(t), 4);
       mbar_init(bar_pv(t), 1);
     }
+    mbar_init(bar_qempty, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -274,85 +303,122 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
   if (warp < 8) {
     regs_inc<PAIR_REGS_NORM>();
     // normalizer warpgroups: see prefill_pair_normalizer above
-    prefill_pair_normalizer<D, KST, VST, CAP>(A, smem, tmem, warp, lane, q0, bh0, kb0, nblk,
-                                         bar_sfull(warp >> 2), bar_pfull(warp >> 2),
-                                         bar_pv(warp >> 2), abort_flag);
-  
+    int g0 = 0;
+    for (int round = 0;; ++round) {
+      const int rank = pair_rank(round, cta, G);
+      if (rank >= ntiles) break;
+      const PairTile T = pair_tile(P, rank);
+      if (!prefill_pair_normalizer<D, KST, VST, CAP>(A, smem, tmem, warp, lane, T.q0, T.bh0,
+                                                      T.kb0, T.nblk, g0, bar_sfull(warp >> 2),
+                                                      bar_pfull(warp >> 2), bar_pv(warp >> 2),
+                                                      abort_flag))
+        break;
+      g0 += T.nblk;
+    }
   } else {
     regs_dec<PAIR_REGS_CTRL>();
-    if (warp == 8) {
-      // ======================= TMA producer ===================================
-      if (lane == 0 && nblk > 0) {
-        tma_prefetch_desc(&tmq);
-        tma_prefetch_desc(&tmk);
-        tma_prefetch_desc(&tmv);
+    if (warp == 8 && lane == 0) {
+      // ======================= TMA producer =================================
+      tma_prefetch_desc(&tmq);
+      tma_prefetch_desc(&tmk);
+      tma_prefetch_desc(&tmv);
+      int g0 = 0, tq = 0;  // blocks and tiles (with blocks) already loaded
+      bool ok = true;
+      for (int round = 0; ok; ++round) {
+        const int rank = pair_rank(round, cta, G);
+        if (rank >= ntiles) break;
+        const PairTile T = pair_tile(P, rank);
+        if (T.nblk == 0) continue;
+        // the previous tile's QK products have read its Q tiles
+        if (tq > 0 && !mbar_wait(bar_qempty, (tq - 1) & 1, abort_flag)) break;
         mbar_expect_tx(bar_q, 2 * LY::QBYTES);
-  #pragma unroll
+#pragma unroll
         for (int t = 0; t < 2; ++t)
-  #pragma unroll
+#pragma unroll
           for (int x = 0; x < D / 64; ++x)
             tma_load_3d(smem_addr(smem + LY::OFF_Q + t * LY::QBYTES + x * TC_BM * 128), &tmq,
-                        bar_q, x * 64, q0, bh0 + t);
-        for (int j = 0; j < nblk; ++j) {
-          const int kb = kb0 + j;
-          const int ks = j % KST;
-          if (j >= KST && !mbar_wait(bar_kempty(ks), ((j / KST) + 1) & 1, abort_flag)) break;
+                        bar_q, x * 64, T.q0, T.bh0 + t);
+        for (int j = 0; j < T.nblk; ++j) {
+          const int gj = g0 + j, kb = T.kb0 + j;
+          const int ks = gj % KST;
+          if (gj >= KST && !mbar_wait(bar_kempty(ks), ((gj / KST) + 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
           mbar_expect_tx(bar_kfull(ks), LY::KBYTES);
           uint8_t* kdst = smem + LY::OFF_K + ks * LY::KBYTES;
-  #pragma unroll
+#pragma unroll
           for (int x = 0; x < D / 64; ++x)
             tma_load_3d(smem_addr(kdst + x * BN * 128), &tmk, bar_kfull(ks), x * 64, kb * BN,
-                        b * P.Hkv + g);
-          const int vs = j % VST;
-          if (j >= VST && !mbar_wait(bar_vempty(vs), ((j / VST) + 1) & 1, abort_flag)) break;
+                        T.b * P.Hkv + T.g);
+          const int vs = gj % VST;
+          if (gj >= VST && !mbar_wait(bar_vempty(vs), ((gj / VST) + 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
           mbar_expect_tx(bar_vfull(vs), LY::VBYTES);
           uint8_t* vdst = smem + LY::OFF_V + vs * LY::VBYTES;
-  #pragma unroll
+#pragma unroll
           for (int x = 0; x < D / 64; ++x)
             tma_load_3d(smem_addr(vdst + x * BN * 128), &tmv, bar_vfull(vs), x * 64, kb * BN,
-                        b * P.Hkv + g);
+                        T.b * P.Hkv + T.g);
         }
+        g0 += T.nblk;
+        ++tq;
       }
-    } else if (warp == 9) {
-      // ======================= MMA issuer =====================================
-      if (lane == 0 && nblk > 0) {
-        constexpr uint32_t IDESC_S = idesc_bf16(TC_BM, BN, 0, 0);
-        constexpr uint32_t IDESC_O = idesc_bf16(TC_BM, D, 0, 1);
-        bool ok = mbar_wait_spin(bar_q, 0, abort_flag);
+    } else if (warp == 9 && lane == 0) {
+      // ======================= MMA issuer ===================================
+      constexpr uint32_t IDESC_S = idesc_bf16(TC_BM, BN, 0, 0);
+      constexpr uint32_t IDESC_O = idesc_bf16(TC_BM, D, 0, 1);
+      auto issue_qk = [&](int t, int gj) {
+        const uint32_t qbase = smem_addr(smem + LY::OFF_Q + t * LY::QBYTES);
+        const uint32_t kbase = smem_addr(smem + LY::OFF_K + (gj % KST) * LY::KBYTES);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad =
+              sdesc_sw128(qbase + (kk >> 2) * TC_BM * 128 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(kbase + (kk >> 2) * BN * 128 + (kk & 3) * 32, 16, 1024);
+          umma_ss(tmem + LY::TM_S + t * BN, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar_sfull(t));
+      };
+      int g0 = 0, tq = 0;
+      bool ok = true;
+      for (int round = 0; ok; ++round) {
+        const int rank = pair_rank(round, cta, G);
+        if (rank >= ntiles) break;
+        const PairTile T = pair_tile(P, rank);
+        const int nblk = T.nblk;
+        if (nblk == 0) continue;
+        ok = mbar_wait_spin(bar_q, tq & 1, abort_flag);
         tc_fence_after();
-        auto issue_qk = [&](int t, int j) {
-          const uint32_t qbase = smem_addr(smem + LY::OFF_Q + t * LY::QBYTES);
-          const uint32_t kbase = smem_addr(smem + LY::OFF_K + (j % KST) * LY::KBYTES);
-  #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ad =
-                sdesc_sw128(qbase + (kk >> 2) * TC_BM * 128 + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(kbase + (kk >> 2) * BN * 128 + (kk & 3) * 32, 16, 1024);
-            umma_ss(tmem + LY::TM_S + t * BN, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(bar_sfull(t));
-        };
-        // prologue: both tiles' scores of the first block
-        if (ok && mbar_wait_spin(bar_kfull(0), 0, abort_flag)) {
+        // prologue: both tiles' scores of the first block (S of either tile
+        // held the previous tile's last P, whose PV was issued before)
+        if (ok && mbar_wait_spin(bar_kfull(g0 % KST), (g0 / KST) & 1, abort_flag)) {
           tc_fence_after();
-          issue_qk(0, 0);
-          issue_qk(1, 0);
-          umma_commit(bar_kempty(0));
+          issue_qk(0, g0);
+          issue_qk(1, g0);
+          umma_commit(bar_kempty(g0 % KST));
+          if (nblk == 1) umma_commit(bar_qempty);
         } else {
           ok = false;
         }
         for (int j = 0; ok && j < nblk; ++j) {
-          const int vs = j % VST;
-          if (!mbar_wait_spin(bar_vfull(vs), (j / VST) & 1, abort_flag)) break;
+          const int gj = g0 + j;
+          const int vs = gj % VST;
+          if (!mbar_wait_spin(bar_vfull(vs), (gj / VST) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
           bool k_next = false;
           for (int t = 0; t < 2; ++t) {
-            if (!mbar_wait_spin(bar_pfull(t), j & 1, abort_flag)) {
+            if (!mbar_wait_spin(bar_pfull(t), gj & 1, abort_flag)) {
               ok = false;
               break;
             }
             tc_fence_after();
             const uint32_t vbase = smem_addr(smem + LY::OFF_V + vs * LY::VBYTES);
-  #pragma unroll
+#pragma unroll
             for (int kk = 0; kk < BN / 16; ++kk) {
               // V block [BN keys][D] in 64-column boxes: MN-major B operand
               const uint64_t bd = sdesc_sw128(vbase + kk * 16 * 128, BN * 128, 1024);
@@ -364,18 +430,24 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
             if (j + 1 < nblk) {
               // this tile's next scores go in behind its PV (issue order)
               if (t == 0) {
-                if (!mbar_wait_spin(bar_kfull((j + 1) % KST), ((j + 1) / KST) & 1, abort_flag)) {
+                if (!mbar_wait_spin(bar_kfull((gj + 1) % KST), ((gj + 1) / KST) & 1,
+                                    abort_flag)) {
                   ok = false;
                   break;
                 }
                 tc_fence_after();
                 k_next = true;
               }
-              issue_qk(t, j + 1);
-              if (t == 1 && k_next) umma_commit(bar_kempty((j + 1) % KST));
+              issue_qk(t, gj + 1);
+              if (t == 1 && k_next) {
+                umma_commit(bar_kempty((gj + 1) % KST));
+                if (j + 2 == nblk) umma_commit(bar_qempty);
+              }
             }
           }
         }
+        g0 += nblk;
+        ++tq;
       }
     }
   }
