@@ -42,6 +42,7 @@ then masked; query head ``h`` reads key/value head ``h // (Hq // Hkv)``.
 from .attention import (  # noqa: F401
     NORMALIZERS,
     allowed_matrix,
+    block_allowed,
     transform_scores,
     softmax_row,
     softmax1_row,

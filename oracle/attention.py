@@ -47,6 +47,19 @@ def allowed_matrix(Tq, Tk, causal, window):
     return ok
 
 
+BLOCK = 128  # side of one block of a block mask
+
+
+def block_allowed(block_mask_bh, Tq, Tk):
+    """Boolean [Tq, Tk] of one (batch, head) block mask: a block mask keeps or
+    drops whole 128 x 128 blocks of (query, key) pairs ("Attention variants",
+    TensorCAD, section "C. Keep the fused kernel": a mask also yields a block
+    mask, and whole blocks that are masked out are skipped).
+    ``block_mask_bh`` is [ceil(Tq/128), ceil(Tk/128)], nonzero = keep."""
+    bm = np.asarray(block_mask_bh) != 0
+    return bm[np.arange(Tq)[:, None] // BLOCK, np.arange(Tk)[None, :] // BLOCK]
+
+
 def transform_scores(s, scale, softcap):
     """Scale the raw dot products, then apply the logit soft-cap.
 
@@ -196,7 +209,7 @@ def _f64(x):
 
 
 def attention_rows(q, k, v, rows, scale, normalizer, causal=False, window=0,
-                   softcap=0.0, want_weights=False, sinks=None):
+                   softcap=0.0, want_weights=False, sinks=None, block_mask=None):
     """Attention output for selected query rows.
 
     ``q`` [B, Hq, Tq, d], ``k`` [B, Hkv, Tk, d], ``v`` [B, Hkv, Tk, dv]
@@ -209,7 +222,9 @@ def attention_rows(q, k, v, rows, scale, normalizer, causal=False, window=0,
 
     ``sinks`` (length Hq, natural-log logits) turns softmax into softmax
     with a learned per-head sink (``softmax_sink_row``); only with
-    ``normalizer == "softmax"``.
+    ``normalizer == "softmax"``.  ``block_mask`` ([B, Hq, ceil(Tq/128),
+    ceil(Tk/128)], nonzero = keep) removes whole 128 x 128 blocks on top of
+    the causal / window rule (``block_allowed``).
 
     Returns ``out`` [n, dv], ``row_stat`` [n] and, if asked, dense weights
     [n, Tk] with exact zeros on masked keys.
@@ -237,8 +252,10 @@ def attention_rows(q, k, v, rows, scale, normalizer, causal=False, window=0,
         qi = rows[sel, 2]
         s = q[b, h, qi, :] @ k[b, g].T            # [len(sel), Tk]
         z = transform_scores(s, scale, softcap)
+        ok_bh = ok_all if block_mask is None else \
+            ok_all & block_allowed(block_mask[b, h], Tq, Tk)
         for t, (r, i) in enumerate(zip(sel, qi)):
-            ok = ok_all[i]
+            ok = ok_bh[i]
             if sinks is None:
                 p, st = normalize_row(z[t][ok], normalizer)
             else:
@@ -252,7 +269,7 @@ def attention_rows(q, k, v, rows, scale, normalizer, causal=False, window=0,
 
 
 def attention_fwd(q, k, v, scale, normalizer, causal=False, window=0,
-                  softcap=0.0, want_weights=False, sinks=None):
+                  softcap=0.0, want_weights=False, sinks=None, block_mask=None):
     """Full attention forward: ``out`` [B, Hq, Tq, dv], ``row_stat``
     [B, Hq, Tq] and optionally ``weights`` [B, Hq, Tq, Tk] (float64)."""
     qa = _f64(q)
@@ -262,7 +279,8 @@ def attention_fwd(q, k, v, scale, normalizer, causal=False, window=0,
                              indexing="ij")
     rows = np.stack([bb.ravel(), hh.ravel(), ii.ravel()], axis=1)
     out, stat, w = attention_rows(qa, k, v, rows, scale, normalizer, causal,
-                                  window, softcap, want_weights, sinks)
+                                  window, softcap, want_weights, sinks,
+                                  block_mask)
     dv = out.shape[1]
     out = out.reshape(B, Hq, Tq, dv)
     stat = stat.reshape(B, Hq, Tq)
