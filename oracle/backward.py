@@ -33,8 +33,8 @@ matrix products, with grouped-query heads summed into their key/value head.
 
 import numpy as np
 
-from .attention import (_f64, allowed_matrix, normalize_row, softmax_sink_row,
-                        transform_scores)
+from .attention import (_f64, allowed_matrix, block_allowed, normalize_row,
+                        softmax_sink_row, transform_scores)
 
 
 def row_vjp(p, g, normalizer):
@@ -56,13 +56,14 @@ def row_vjp(p, g, normalizer):
 
 
 def attention_bwd(q, k, v, dout, scale, normalizer, causal=False, window=0,
-                  softcap=0.0, sinks=None):
+                  softcap=0.0, sinks=None, block_mask=None):
     """Gradients ``(dq, dk, dv)`` of ``L = sum(dout * O)`` for the forward of
     ``attention_fwd`` with the same arguments.  Shapes as in the forward:
     ``q`` [B, Hq, Tq, d], ``k`` [B, Hkv, Tk, d], ``v`` [B, Hkv, Tk, dv],
     ``dout`` [B, Hq, Tq, dv]; query head ``h`` reads key/value head
     ``h // (Hq // Hkv)``, so ``dk`` and ``dv`` sum over the heads of a group.
-    ``sinks`` (length Hq) only with softmax.  Returns float64 arrays."""
+    ``sinks`` (length Hq) only with softmax; ``block_mask`` as in the
+    forward.  Returns float64 arrays."""
     q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
     B, Hq, Tq, d = q.shape
     _, Hkv, Tk, _ = k.shape
@@ -83,11 +84,13 @@ def attention_bwd(q, k, v, dout, scale, normalizer, causal=False, window=0,
                 dzds = scale * (1.0 - np.tanh(scale * s / softcap) ** 2)
             else:
                 dzds = np.full_like(s, scale)
+            ok_bh = ok if block_mask is None else \
+                ok & block_allowed(block_mask[b, h], Tq, Tk)
             P = np.zeros((Tq, Tk))
             dZ = np.zeros((Tq, Tk))
             dP = dout[b, h] @ v[b, g].T                  # dL/dp
             for i in range(Tq):
-                m = ok[i]
+                m = ok_bh[i]
                 if sinks is None:
                     p, _ = normalize_row(z[i][m], normalizer)
                 else:

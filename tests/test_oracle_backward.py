@@ -142,3 +142,32 @@ def test_planted_backward_mistakes_are_caught(normalizer, mistake, monkeypatch):
     monkeypatch.setattr(bwd, "row_vjp", mistake)
     bad = bwd.attention_bwd(q, k, v, dout, 0.9, normalizer, True)
     assert max(np.abs(g - w).max() for g, w in zip(bad, want)) > 1e-3
+
+
+@pytest.mark.parametrize("normalizer", NORMS)
+def test_backward_with_block_mask_matches_finite_differences(normalizer):
+    """A block mask drops whole 128 x 128 blocks: central differences of the
+    forward oracle on a sample of coordinates of q, k and v."""
+    rng = np.random.default_rng(23)
+    B, Hq, Hkv, T, d = 1, 2, 1, 260, 3
+    q = rng.normal(size=(B, Hq, T, d)) * 1.5
+    k = rng.normal(size=(B, Hkv, T, d)) * 1.5
+    v = rng.normal(size=(B, Hkv, T, d))
+    dout = rng.normal(size=(B, Hq, T, d))
+    bm = np.array([[[[1, 0, 1], [0, 1, 1], [1, 1, 0]],
+                    [[1, 1, 1], [1, 0, 1], [0, 1, 1]]]], dtype=np.uint8)
+    got = bwd.attention_bwd(q, k, v, dout, 0.8, normalizer, True, block_mask=bm)
+
+    def loss(q_, k_, v_):
+        o, _, _ = attention_fwd(q_, k_, v_, 0.8, normalizer, True, block_mask=bm)
+        return float((o * dout).sum())
+    eps = 1e-6
+    for which, x in enumerate((q, k, v)):
+        for _ in range(12):
+            idx = tuple(int(rng.integers(0, n)) for n in x.shape)
+            base = [q.copy(), k.copy(), v.copy()]
+            base[which][idx] += eps
+            lp = loss(*base)
+            base[which][idx] -= 2 * eps
+            lm = loss(*base)
+            assert abs((lp - lm) / (2 * eps) - got[which][idx]) < 2e-7
