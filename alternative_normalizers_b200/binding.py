@@ -40,6 +40,7 @@ class NattnArgs(ctypes.Structure):
         ("num_pages", ctypes.c_int),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("stream", ctypes.c_void_p), ("sinks", ctypes.c_void_p),
+        ("block_mask", ctypes.c_void_p),
     ]
 
 
@@ -59,7 +60,7 @@ class NattnBwdArgs(ctypes.Structure):
         ("causal", ctypes.c_int), ("window", ctypes.c_int),
         ("softcap", ctypes.c_float), ("sinks", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
-        ("stream", ctypes.c_void_p),
+        ("stream", ctypes.c_void_p), ("block_mask", ctypes.c_void_p),
     ]
 
 
@@ -182,11 +183,13 @@ def _norm_id(normalizer):
 def build_args(q, k, v, out, row_stat=None, weights=None, *, normalizer,
                causal=False, window=0, softcap=0.0, scale=None,
                block_table=None, seqlens=None, page_size=0, max_seqlen=None,
-               stream=None, row_nnz=None, sinks=None):
+               stream=None, row_nnz=None, sinks=None, block_mask=None):
     """Fill an ``NattnArgs`` from torch tensors (no device work).
     ``row_nnz`` (int32 [B, Hq, Tq] or None) receives the number of keys with
     a nonzero weight in each row; ``sinks`` (float32 [Hq] or None) are the
-    learned per-head sink logits (softmax only)."""
+    learned per-head sink logits (softmax only); ``block_mask`` (uint8
+    [B, Hq, ceil(Tq/128), ceil(Tk/128)] or None) drops whole 128 x 128
+    blocks of (query, key) pairs."""
     import torch
     B, Hq, Tq, d = q.shape
     a = NattnArgs()
@@ -194,6 +197,7 @@ def build_args(q, k, v, out, row_stat=None, weights=None, *, normalizer,
     a.row_stat, a.weights = _ptr(row_stat), _ptr(weights)
     a.row_nnz = _ptr(row_nnz)
     a.sinks = _ptr(sinks)
+    a.block_mask = _ptr(block_mask)
     a.B, a.Hq, a.Tq, a.d = B, Hq, Tq, d
     a.Hkv = k.shape[1]
     a.dv = v.shape[3]
@@ -229,11 +233,13 @@ def _run(a, workspace_holder):
 
 def attention(q, k, v, normalizer="softmax", causal=False, window=0,
               softcap=0.0, scale=None, want_weights=False, out=None,
-              row_stat=None, row_nnz=None, sinks=None):
+              row_stat=None, row_nnz=None, sinks=None, block_mask=None):
     """Dense attention forward.  q [B,Hq,Tq,d], k [B,Hkv,Tk,d], v
     [B,Hkv,Tk,dv] (bf16, CUDA, contiguous).  Returns (out, row_stat,
     weights|None); fills ``row_nnz`` (int32 [B,Hq,Tq]) when given.
-    ``sinks`` (float32 [Hq], softmax only): learned per-head sink logits."""
+    ``sinks`` (float32 [Hq], softmax only): learned per-head sink logits.
+    ``block_mask`` (uint8 [B, Hq, ceil(Tq/128), ceil(Tk/128)]): 0 drops the
+    128 x 128 block of (query, key) pairs."""
     import torch
     B, Hq, Tq, _ = q.shape
     Tk, dv = k.shape[2], v.shape[3]
@@ -245,7 +251,7 @@ def attention(q, k, v, normalizer="softmax", causal=False, window=0,
                           device=q.device) if want_weights else None
     a = build_args(q, k, v, out, row_stat, weights, normalizer=normalizer,
                    causal=causal, window=window, softcap=softcap, scale=scale,
-                   row_nnz=row_nnz, sinks=sinks)
+                   row_nnz=row_nnz, sinks=sinks, block_mask=block_mask)
     keep = []
     _run(a, keep)
     return out, row_stat, weights
@@ -277,7 +283,7 @@ def paged_attention(q, k_pool, v_pool, block_table, seqlens, max_seqlen,
 
 def build_bwd_args(q, k, v, out, row_stat, grad_out, grad_q, grad_k, grad_v, *,
                    normalizer, causal=False, window=0, softcap=0.0,
-                   scale=None, sinks=None, stream=None):
+                   scale=None, sinks=None, stream=None, block_mask=None):
     """Fill an ``NattnBwdArgs`` from torch tensors (no device work)."""
     import torch
     B, Hq, Tq, d = q.shape
@@ -291,6 +297,7 @@ def build_bwd_args(q, k, v, out, row_stat, grad_out, grad_q, grad_k, grad_v, *,
     a.normalizer = _norm_id(normalizer)
     a.causal, a.window, a.softcap = int(bool(causal)), int(window), float(softcap)
     a.sinks = _ptr(sinks)
+    a.block_mask = _ptr(block_mask)
     if stream is None and q.is_cuda:
         stream = torch.cuda.current_stream(q.device).cuda_stream
     a.stream = stream
@@ -299,7 +306,7 @@ def build_bwd_args(q, k, v, out, row_stat, grad_out, grad_q, grad_k, grad_v, *,
 
 def attention_backward(q, k, v, out, row_stat, grad_out, normalizer="softmax",
                        causal=False, window=0, softcap=0.0, scale=None,
-                       sinks=None):
+                       sinks=None, block_mask=None):
     """Gradients (dq, dk, dv) of sum(grad_out * O) for the dense forward
     that produced ``out`` and ``row_stat`` with the same arguments (bf16,
     CUDA, contiguous; d == dv in {64, 128})."""
@@ -307,7 +314,8 @@ def attention_backward(q, k, v, out, row_stat, grad_out, normalizer="softmax",
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     a = build_bwd_args(q, k, v, out, row_stat, grad_out, dq, dk, dv,
                        normalizer=normalizer, causal=causal, window=window,
-                       softcap=softcap, scale=scale, sinks=sinks)
+                       softcap=softcap, scale=scale, sinks=sinks,
+                       block_mask=block_mask)
     need = nattn_bwd_workspace_size(a)
     ws = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     a.workspace, a.workspace_bytes = ws.data_ptr(), need

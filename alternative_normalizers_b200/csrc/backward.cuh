@@ -351,7 +351,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const int jb = (kb0 + j) * BN;
       const int kl = rr.lo - jb;
       const unsigned span = rr.hi >= rr.lo ? (unsigned)(rr.hi - rr.lo) : 0u;
-      const bool any = rr.hi >= rr.lo;
+      // a block the block mask drops counts as masked whole
+      const bool any = rr.hi >= rr.lo && block_kept(P, b, h, qt, jb >> 7);
       uint32_t pk[32];
 #pragma unroll
       for (int k = 0; k < BN; k += 2) {
@@ -668,7 +669,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       // visible query columns of this key: [cl, cl + span]
       const int cl = qr.lo - q0;
       const unsigned span = qr.hi >= qr.lo ? (unsigned)(qr.hi - qr.lo) : 0u;
-      const bool any = qr.hi >= qr.lo;
+      // a block the block mask drops counts as masked whole
+      const bool any = qr.hi >= qr.lo && block_kept(P, b, h, q0 >> 7, kt);
       uint32_t ppk[32], dpk[32];
 #pragma unroll
       for (int c4 = 0; c4 < BQ; c4 += 4) {

@@ -178,7 +178,7 @@ int validate(const nattn_args* a) {
     if (!a->seqlens || a->page_size < 1 || a->block_table_stride < 1 || a->num_pages < 1 ||
         a->Tk < 1)
       return NATTN_EINVAL;
-    if (a->weights) return NATTN_EUNSUPPORTED;
+    if (a->weights || a->block_mask) return NATTN_EUNSUPPORTED;
     if ((long long)a->num_pages * a->Hkv * a->page_size >= (1ll << 31))
       return NATTN_ETOOLARGE;
   } else {
@@ -289,6 +289,9 @@ Problem to_problem(const nattn_args* a) {
   P.window = a->window;
   P.softcap = a->softcap;
   P.sinks = a->sinks;
+  P.block_mask = a->block_mask;
+  P.bm_nq = (a->Tq + 127) / 128;
+  P.bm_nk = (a->Tk + 127) / 128;
   P.block_table = a->block_table;
   P.seqlens = a->seqlens;
   P.page_size = a->page_size;
@@ -606,6 +609,7 @@ int validate_bwd(const nattn_bwd_args* a) {
   f.window = a->window;
   f.softcap = a->softcap;
   f.sinks = a->sinks;
+  f.block_mask = a->block_mask;
   f.row_stat = const_cast<float*>(a->row_stat);
   int rc = validate(&f);
   if (rc != NATTN_OK) return rc;
@@ -690,6 +694,9 @@ int launch_bwd(const nattn_bwd_args* a, cudaStream_t st) {
   P.window = a->window;
   P.softcap = a->softcap;
   P.sinks = a->sinks;
+  P.block_mask = a->block_mask;
+  P.bm_nq = (a->Tq + 127) / 128;
+  P.bm_nk = (a->Tk + 127) / 128;
   A.dout = static_cast<const bf16*>(a->grad_out);
   A.dq = static_cast<bf16*>(a->grad_q);
   A.dk = static_cast<bf16*>(a->grad_k);

@@ -62,7 +62,7 @@ struct PairLayout {
 // One unit of work: the same 128 query rows of the two query heads h0, h0 + 1
 // (one GQA group) of batch b, and the visible key blocks [kb0, kb0 + nblk).
 struct PairTile {
-  int b, h0, g, bh0, q0, kb0, nblk;
+  int b, h0, g, bh0, q0, kb0, kend, nblk;  // nblk: blocks in [kb0, kend) a block mask keeps
 };
 
 // Tile of heaviest-first rank `rank`: under the causal mask the last query
@@ -85,7 +85,8 @@ __device__ __forceinline__ PairTile pair_tile(const Problem& P, int rank) {
   const int klo = max(0, r_first.lo);
   const int khi = min(P.Tk - 1, r_last.hi);
   T.kb0 = klo / 128;
-  T.nblk = (khi >= klo) ? (khi / 128 - T.kb0 + 1) : 0;
+  T.kend = (khi >= klo) ? khi / 128 + 1 : T.kb0;
+  T.nblk = count_kept<128>(P, T.b, T.h0, T.h0 + 1, qt, T.kb0, T.kend);
   return T;
 }
 
@@ -104,8 +105,8 @@ __device__ __forceinline__ int pair_rank(int round, int c, int G) {
 // across tiles.  Returns false if a wait gave up.
 template <int D, int KST, int VST, bool CAP>
 __device__ __forceinline__ bool prefill_pair_normalizer(
-    const TcArgs& A, uint8_t* smem, uint32_t tmem, int warp, int lane, int q0, int bh0,
-    int kb0, int nblk, int g0, uint32_t bar_sf, uint32_t bar_pf, uint32_t bar_pvt,
+    const TcArgs& A, uint8_t* smem, uint32_t tmem, int warp, int lane, int b, int q0, int bh0,
+    int kb0, int kend, int nblk, int g0, uint32_t bar_sf, uint32_t bar_pf, uint32_t bar_pvt,
     volatile int* abort_flag) {
   using LY = PairLayout<D, KST, VST>;
   constexpr int BN = LY::BN;
@@ -131,6 +132,11 @@ __device__ __forceinline__ bool prefill_pair_normalizer(
   float m_run = sink2;
   float l_run = (sink2 == -INFINITY) ? 0.f : 1.f;
   bool alive = true;
+  // block mask: the pair walks the blocks either head keeps; a block this
+  // tile's head drops is masked whole
+  const int qb = q0 >> 7, hp = bh0 % P.Hq, hown = hp + t;
+  int kb = next_kept<BN>(P, b, hp, hp + 1, qb, kb0, kend);
+  int nvis = 0;  // visible keys in kept blocks (row_nnz)
 
   for (int j = 0; j < nblk; ++j) {
     if (!__all_sync(0xffffffffu, mbar_wait_spin(bar_sf, (g0 + j) & 1, abort_flag))) {
@@ -138,14 +144,18 @@ __device__ __forceinline__ bool prefill_pair_normalizer(
       break;
     }
     tc_fence_after();
-    const int jb = (kb0 + j) * BN;
-    const bool edge = !(rr.lo <= jb && rr.hi >= jb + BN - 1);
+    const int jb = kb * BN;
+    const bool own = block_kept(P, b, hown, qb, kb);
+    const bool edge = !own || !(rr.lo <= jb && rr.hi >= jb + BN - 1);
     int kl = rr.lo - jb;
     unsigned span = (unsigned)(rr.hi - rr.lo);
-    if (rr.hi < rr.lo) {
+    if (rr.hi < rr.lo || !own) {
       kl = BN;
       span = 0;
+    } else {
+      nvis += max(0, min(rr.hi, jb + BN - 1) - max(rr.lo, jb) + 1);
     }
+    kb = next_kept<BN>(P, b, hp, hp + 1, qb, kb + 1, kend);
     // the whole S row (128 scores) in registers: one TMEM read per block;
     // x is the raw score on the fast path, else z in log2 units; masked
     // entries -inf
@@ -236,7 +246,8 @@ __device__ __forceinline__ bool prefill_pair_normalizer(
     }
   }
   if (row_ok && P.row_stat) P.row_stat[flat] = stat;
-  if (row_ok && P.row_nnz) P.row_nnz[flat] = rr.hi >= rr.lo ? rr.hi - rr.lo + 1 : 0;
+  if (row_ok && P.row_nnz)
+    P.row_nnz[flat] = P.block_mask ? nvis : (rr.hi >= rr.lo ? rr.hi - rr.lo + 1 : 0);
   return alive;
 }
 
@@ -308,8 +319,9 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
       const int rank = pair_rank(round, cta, G);
       if (rank >= ntiles) break;
       const PairTile T = pair_tile(P, rank);
-      if (!prefill_pair_normalizer<D, KST, VST, CAP>(A, smem, tmem, warp, lane, T.q0, T.bh0,
-                                                      T.kb0, T.nblk, g0, bar_sfull(warp >> 2),
+      if (!prefill_pair_normalizer<D, KST, VST, CAP>(A, smem, tmem, warp, lane, T.b, T.q0,
+                                                      T.bh0, T.kb0, T.kend, T.nblk, g0,
+                                                      bar_sfull(warp >> 2),
                                                       bar_pfull(warp >> 2), bar_pv(warp >> 2),
                                                       abort_flag))
         break;
@@ -338,8 +350,10 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
           for (int x = 0; x < D / 64; ++x)
             tma_load_3d(smem_addr(smem + LY::OFF_Q + t * LY::QBYTES + x * TC_BM * 128), &tmq,
                         bar_q, x * 64, T.q0, T.bh0 + t);
-        for (int j = 0; j < T.nblk; ++j) {
-          const int gj = g0 + j, kb = T.kb0 + j;
+        int kb = next_kept<BN>(P, T.b, T.h0, T.h0 + 1, T.q0 >> 7, T.kb0, T.kend);
+        for (int j = 0; j < T.nblk; ++j, kb = next_kept<BN>(P, T.b, T.h0, T.h0 + 1, T.q0 >> 7,
+                                                            kb + 1, T.kend)) {
+          const int gj = g0 + j;
           const int ks = gj % KST;
           if (gj >= KST && !mbar_wait(bar_kempty(ks), ((gj / KST) + 1) & 1, abort_flag)) {
             ok = false;

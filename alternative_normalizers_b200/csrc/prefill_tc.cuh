@@ -226,7 +226,9 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
   const int klo = max(0, r_first.lo);
   const int khi = min(P.Tk - 1, r_last.hi);
   const int kb0 = klo / BN;
-  const int nblk = (khi >= klo) ? (khi / BN - kb0 + 1) : 0;
+  const int kend = (khi >= klo) ? khi / BN + 1 : kb0;
+  // blocks of [kb0, kend) the block mask keeps (all of them without one)
+  const int nblk = count_kept<BN>(P, b, h, h, qt, kb0, kend);
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + LY::OFF_BAR);
   const uint32_t bar_q = smem_addr(&bars[0]);
@@ -282,8 +284,8 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
       for (int x = 0; x < D / 64; ++x)
         tma_load_3d(smem_addr(smem + LY::OFF_Q + x * TC_BM * 128), &tmq, bar_q, x * 64, q0,
                     bh);
-      for (int j = 0; j < nblk; ++j) {
-        const int kb = kb0 + j;
+      int kb = next_kept<BN>(P, b, h, h, qt, kb0, kend);
+      for (int j = 0; j < nblk; ++j, kb = next_kept<BN>(P, b, h, h, qt, kb + 1, kend)) {
         const int ks = j % KST;
         if (j >= KST && !mbar_wait(bar_kempty(ks), ((j / KST) + 1) & 1, abort_flag)) break;
         mbar_expect_tx(bar_kfull(ks), LY::KBYTES);
@@ -411,14 +413,15 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
     const bool entmax = P.norm == NATTN_ENTMAX15;
     bool alive = true;
 
-    for (int j = 0; j < nblk; ++j) {
+    int kbc = next_kept<BN>(P, b, h, h, qt, kb0, kend);  // key block of step j
+    for (int j = 0; j < nblk; ++j, kbc = next_kept<BN>(P, b, h, h, qt, kbc + 1, kend)) {
       const int sb = j % NSB;
       if (!__all_sync(0xffffffffu, mbar_wait_spin(bar_sfull(sb), (j / NSB) & 1, abort_flag))) {
         alive = false;
         break;
       }
       tc_fence_after();
-      const int jb = (kb0 + j) * BN + cbase;  // first key of this thread's columns
+      const int jb = kbc * BN + cbase;  // first key of this thread's columns
       const bool edge = !(rr.lo <= jb && rr.hi >= jb + NC - 1);
       // visible keys of this row relative to jb: [klb, klb + span]
       int klb = rr.lo - jb;
@@ -745,8 +748,19 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
       }
       if (row_ok && P.row_stat && half == 0) P.row_stat[flat] = stat;
       if constexpr (MODE == TC_ONLINE) {
-        if (row_ok && P.row_nnz && half == 0)
-          P.row_nnz[flat] = rr.hi >= rr.lo ? rr.hi - rr.lo + 1 : 0;
+        if (row_ok && P.row_nnz && half == 0) {
+          int n = 0;
+          if (rr.hi >= rr.lo) {
+            if (P.block_mask == nullptr) {
+              n = rr.hi - rr.lo + 1;
+            } else {
+              for (int kb = kb0; kb < kend; ++kb)
+                if (block_kept(P, b, h, qt, (kb * BN) >> 7))
+                  n += max(0, min(rr.hi, kb * BN + BN - 1) - max(rr.lo, kb * BN) + 1);
+            }
+          }
+          P.row_nnz[flat] = n;
+        }
       }
     }
   }

@@ -24,6 +24,10 @@ struct Problem {
   // learned per-head attention sinks: logit of a value-0 sink in the
   // softmax denominator of query head h (natural-log units), or null
   const float* sinks;
+  // block mask [B, Hq, bm_nq, bm_nk] (nonzero = keep the 128 x 128 block of
+  // (query, key) pairs) or null; bm_nq = ceil(Tq / 128), bm_nk = ceil(Tk / 128)
+  const uint8_t* block_mask;
+  int bm_nq, bm_nk;
   // paged mode (block_table != nullptr)
   const int32_t* block_table;
   const int32_t* seqlens;
@@ -66,6 +70,40 @@ __device__ __forceinline__ RowRange row_range(const Problem& P, int i, int L) {
 __device__ __forceinline__ float sink_logit(const Problem& P, int h) {
   if (P.sinks != nullptr) return P.sinks[h];
   return P.norm == NATTN_SOFTMAX1 ? 0.f : -INFINITY;
+}
+
+// Block mask: is the 128 x 128 block (query block qb, key block kb) of query
+// head h of batch b kept?  Whole blocks that a mask drops are skipped
+// ("Attention variants", TensorCAD, section "C. Keep the fused kernel": a
+// mask yields a block mask, and masked-out blocks are skipped).  Always true
+// without a block mask.
+__device__ __forceinline__ bool block_kept(const Problem& P, int b, int h, int qb, int kb) {
+  if (P.block_mask == nullptr) return true;
+  return P.block_mask[(((size_t)b * P.Hq + h) * P.bm_nq + qb) * P.bm_nk + kb] != 0;
+}
+
+// Key blocks of BN keys (BN = 64 or 128) in [kb, kend) that heads h0 or h1
+// keep for query block qb: the next one at or after kb, and how many there
+// are.  Every role of a kernel walks the same sequence.
+template <int BN>
+__device__ __forceinline__ int next_kept(const Problem& P, int b, int h0, int h1, int qb, int kb,
+                                         int kend) {
+  if (P.block_mask == nullptr) return kb;
+  while (kb < kend && !block_kept(P, b, h0, qb, (kb * BN) >> 7) &&
+         !block_kept(P, b, h1, qb, (kb * BN) >> 7))
+    ++kb;
+  return kb;
+}
+template <int BN>
+__device__ __forceinline__ int count_kept(const Problem& P, int b, int h0, int h1, int qb, int kb,
+                                          int kend) {
+  if (P.block_mask == nullptr) return kend - kb;
+  int n = 0;
+  for (; kb < kend; ++kb)
+    n += (block_kept(P, b, h0, qb, (kb * BN) >> 7) || block_kept(P, b, h1, qb, (kb * BN) >> 7))
+             ? 1
+             : 0;
+  return n;
 }
 
 // Address of key (or value) row j of sequence b, kv head g.  Dense layout

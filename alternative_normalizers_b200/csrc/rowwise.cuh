@@ -220,6 +220,8 @@ __global__ void __launch_bounds__(ROW_THREADS)
           if (sub == 0 && jj < n) {
             float z = s * P.scale;
             if (P.softcap > 0.f) z = P.softcap * tanhf(z / P.softcap);
+            // a key in a block the block mask drops is not visible
+            if (!block_kept(P, b, h, i >> 7, (rr.lo + jj) >> 7)) z = -INFINITY;
             sc[jj] = z * uscale;
           }
         }
@@ -233,7 +235,14 @@ __global__ void __launch_bounds__(ROW_THREADS)
 
     // normalizer: overwrite scores with weights
     float stat;
-    int nnz = n;  // softmax / softmax1: every visible key
+    // softmax / softmax1: every visible key (of the blocks a block mask keeps)
+    int nnz = n;
+    if (P.block_mask != nullptr && n > 0) {
+      nnz = 0;
+      for (int kb = rr.lo >> 7; kb <= (rr.hi >> 7); ++kb)
+        if (block_kept(P, b, h, i >> 7, kb))
+          nnz += min(rr.hi, kb * 128 + 127) - max(rr.lo, kb * 128) + 1;
+    }
     if (P.norm == NATTN_SOFTMAX || P.norm == NATTN_SOFTMAX1) {
       float mx = -INFINITY;
       for (int jj = tid; jj < n; jj += ROW_THREADS) mx = fmaxf(mx, sc[jj]);
@@ -261,7 +270,7 @@ __global__ void __launch_bounds__(ROW_THREADS)
       // runs over the keys within one unit of the maximum, gathered into the
       // column-partials area (free until the PV), unless there are too many
       float tau = INFINITY;
-      if (n > 0) {
+      if (n > 0 && mx != -INFINITY) {  // -inf: every key dropped by the block mask
         float* cand = part;
         constexpr int kCandCap = ROW_WARPS * 256;
         if (tid == 0) s_ncand = 0;

@@ -697,6 +697,33 @@ def detail(args, dev, flush):
         torch.cuda.empty_cache()
     except Exception as exc:
         res["qwen3_8b_prefill_sinks"] = {"error": repr(exc)[:200]}
+    # block mask: the headline shape packed with four causal documents of
+    # 1024 tokens (block-diagonal mask); useful FLOPs = 4 * d per allowed
+    # (query, key) pair, counted exactly
+    try:
+        w = WORKLOADS["qwen3_8b_prefill"]
+        r = Runner(w, dev)
+        doc = 1024 // 128
+        nq = (w.Tq + 127) // 128
+        bm = torch.zeros(w.B, w.Hq, nq, nq, dtype=torch.uint8)
+        for d0 in range(0, nq, doc):
+            bm[..., d0:d0 + doc, d0:d0 + doc] = 1
+        bm = bm.to(dev)
+        for n in w.normalizers:
+            r.args[n].block_mask = bm.data_ptr()
+        per = time_runner(r, max(3, args.steps // 2), 2, flush)
+        pairs = (w.Tq // 1024) * (1024 * 1025 // 2)
+        u = 4.0 * w.d * pairs * w.B * w.Hq
+        vals = {n: round(u / (t * 1e-3) / 1e12, 1) for n, t in per.items()}
+        res["qwen3_8b_prefill_doc_mask"] = {
+            "unit": "useful TFLOP/s (exact allowed pairs)", "value": vals,
+            "ms": {n: round(t, 4) for n, t in per.items()},
+            "roofline_frac": {n: round(v / peaks["bf16_tflops"], 4) for n, v in vals.items()},
+            "roofline_denominator": "of measured bf16_tflops (burst)"}
+        del r, bm
+        torch.cuda.empty_cache()
+    except Exception as exc:
+        res["qwen3_8b_prefill_doc_mask"] = {"error": repr(exc)[:200]}
     return res
 
 

@@ -128,6 +128,19 @@ enum {
  *            the special case sinks[h] = 0.  Any other normalizer with sinks:
  *            NATTN_EUNSUPPORTED.  4-byte aligned (NATTN_EALIGN).
  *
+ * Block mask ("Attention variants: what to open up, and how far",
+ * TensorCAD, section "C. Keep the fused kernel": a mask yields a block mask,
+ * and whole blocks that are masked out are skipped):
+ *   block_mask  uint8 [B, Hq, ceil(Tq/128), ceil(Tk/128)] or NULL, device
+ *            memory.  Entry [b, h, qb, kb] == 0 drops every (query, key)
+ *            pair of query rows [128 qb, 128 qb + 128) and keys
+ *            [128 kb, 128 kb + 128) of query head h, on top of the causal /
+ *            window rule; dropped blocks are neither loaded nor multiplied.
+ *            Document masks (block-aligned documents), block-level prefix-LM
+ *            and block-sparse patterns are block masks.  A row whose visible
+ *            keys are all dropped is a row with no visible key.  Dense mode
+ *            only (paged mode with a block mask: NATTN_EUNSUPPORTED).
+ *
  * window == 0 disables the sliding window; with causal it keeps keys with
  * 0 <= pos - j < window ("attention interface" wiki, section "common
  * flexattention patterns"); without causal it keeps |pos - j| < window.
@@ -157,6 +170,8 @@ typedef struct nattn_args {
   void* stream;             /* cudaStream_t */
   const float* sinks;       /* learned per-head attention sinks, or NULL (see
                                below); NATTN_SOFTMAX only                   */
+  const uint8_t* block_mask;/* 128 x 128 block mask, or NULL (see below);
+                               dense mode only                              */
 } nattn_args;
 
 /*
@@ -240,6 +255,7 @@ typedef struct nattn_bwd_args {
   void* workspace;
   size_t workspace_bytes;
   void* stream;             /* cudaStream_t */
+  const uint8_t* block_mask;/* as in nattn_args                             */
 } nattn_bwd_args;
 
 int nattn_bwd(const nattn_bwd_args* a);
