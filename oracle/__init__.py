@@ -54,5 +54,6 @@ from .attention import (  # noqa: F401
     attention_rows,
     paged_gather,
     paged_decode,
+    varlen_attention,
 )
 from .backward import attention_bwd, row_vjp  # noqa: F401

@@ -290,6 +290,42 @@ def attention_fwd(q, k, v, scale, normalizer, causal=False, window=0,
 
 
 # --------------------------------------------------------------------------
+# Packed variable-length sequences
+# --------------------------------------------------------------------------
+
+def varlen_attention(q, k, v, cu_q, cu_k, scale, normalizer, causal=False,
+                     window=0, softcap=0.0, sinks=None):
+    """Packed variable-length attention ("HF Attention Normalizers", section
+    "Packed Variable-Length Attention": FlashAttention-style packed layouts
+    with cumulative sequence lengths, per-request bottom-right causal
+    alignment, GQA, different query and key lengths).
+
+    ``q`` [total_q, Hq, d], ``k`` [total_k, Hkv, d], ``v`` [total_k, Hkv, dv];
+    sequence ``b`` owns query tokens ``[cu_q[b], cu_q[b+1])`` and key tokens
+    ``[cu_k[b], cu_k[b+1])`` and is an attention problem of its own.  Returns
+    ``out`` [total_q, Hq, dv] and ``row_stat`` [total_q, Hq]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cu_q = np.asarray(cu_q, dtype=np.int64)
+    cu_k = np.asarray(cu_k, dtype=np.int64)
+    total_q, Hq, _ = q.shape
+    dv = v.shape[2]
+    out = np.zeros((total_q, Hq, dv))
+    stat = np.zeros((total_q, Hq))
+    for b in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = cu_q[b], cu_q[b + 1], cu_k[b], cu_k[b + 1]
+        if q1 == q0:
+            continue
+        qs = q[q0:q1].transpose(1, 0, 2)[None]
+        ks = k[k0:k1].transpose(1, 0, 2)[None]
+        vs = v[k0:k1].transpose(1, 0, 2)[None]
+        o, st, _ = attention_fwd(qs, ks, vs, scale, normalizer, causal, window,
+                                 softcap, sinks=sinks)
+        out[q0:q1] = o[0].transpose(1, 0, 2)
+        stat[q0:q1] = st[0].T
+    return out, stat
+
+
+# --------------------------------------------------------------------------
 # Paged KV cache
 # --------------------------------------------------------------------------
 
