@@ -26,6 +26,7 @@ from .binding import (  # noqa: F401
     nattn_version,
     nattn_workspace_size,
     paged_attention,
+    varlen_attention,
 )
 from .workloads import NORMALIZER_IDS, WORKLOADS, Workload  # noqa: F401
 

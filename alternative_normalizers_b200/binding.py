@@ -41,6 +41,8 @@ class NattnArgs(ctypes.Structure):
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("stream", ctypes.c_void_p), ("sinks", ctypes.c_void_p),
         ("block_mask", ctypes.c_void_p),
+        ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_k", ctypes.c_void_p),
+        ("total_q", ctypes.c_int), ("total_k", ctypes.c_int),
     ]
 
 
@@ -255,6 +257,39 @@ def attention(q, k, v, normalizer="softmax", causal=False, window=0,
     keep = []
     _run(a, keep)
     return out, row_stat, weights
+
+
+def varlen_attention(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                     max_seqlen_k, normalizer="softmax", causal=True, window=0,
+                     softcap=0.0, scale=None, sinks=None, out=None,
+                     row_stat=None, row_nnz=None):
+    """Packed variable-length attention: q [total_q, Hq, d], k [total_k,
+    Hkv, d], v [total_k, Hkv, dv] (bf16, CUDA, contiguous), cumulative
+    lengths int32 [B + 1] on the device.  Returns (out [total_q, Hq, dv],
+    row_stat [total_q, Hq]); fills ``row_nnz`` ([total_q, Hq]) when given."""
+    import torch
+    total_q, Hq, d = q.shape
+    total_k, Hkv, _ = k.shape
+    dv = v.shape[2]
+    out = torch.empty(total_q, Hq, dv, dtype=torch.bfloat16, device=q.device) \
+        if out is None else out
+    row_stat = torch.empty(total_q, Hq, dtype=torch.float32, device=q.device) \
+        if row_stat is None else row_stat
+    a = NattnArgs()
+    a.q, a.k, a.v, a.out = _ptr(q), _ptr(k), _ptr(v), _ptr(out)
+    a.row_stat, a.row_nnz, a.sinks = _ptr(row_stat), _ptr(row_nnz), _ptr(sinks)
+    a.B = cu_seqlens_q.numel() - 1
+    a.Hq, a.Hkv, a.d, a.dv = Hq, Hkv, d, dv
+    a.Tq, a.Tk = int(max_seqlen_q), int(max_seqlen_k)
+    a.scale = (1.0 / d ** 0.5) if scale is None else scale
+    a.normalizer = _norm_id(normalizer)
+    a.causal, a.window, a.softcap = int(bool(causal)), int(window), float(softcap)
+    a.cu_seqlens_q, a.cu_seqlens_k = _ptr(cu_seqlens_q), _ptr(cu_seqlens_k)
+    a.total_q, a.total_k = total_q, total_k
+    a.stream = torch.cuda.current_stream(q.device).cuda_stream
+    keep = []
+    _run(a, keep)
+    return out, row_stat
 
 
 def paged_attention(q, k_pool, v_pool, block_table, seqlens, max_seqlen,

@@ -68,6 +68,22 @@ bool make_map_3d(CUtensorMap* m, const void* base, int inner, int rows, long lon
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 tensor in the packed layout [rows][planes][inner] (token-major) with a
+// (64 x 1 x box_rows) box: box_rows rows of one plane, 128-byte swizzle.
+bool make_map_packed(CUtensorMap* m, const void* base, int inner, int planes, long long rows,
+                     int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)planes, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)inner * 2 * planes};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_map_2d(CUtensorMap* m, const void* base, int inner, long long rows, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
@@ -149,6 +165,12 @@ struct Plan {
 };
 
 bool is_paged(const nattn_args* a) { return a->block_table != nullptr; }
+bool is_packed(const nattn_args* a) { return a->cu_seqlens_q != nullptr; }
+
+// Query rows of the problem: B * Hq * Tq, or total_q * Hq when packed.
+long long num_rows(const nattn_args* a) {
+  return is_packed(a) ? (long long)a->total_q * a->Hq : (long long)a->B * a->Hq * a->Tq;
+}
 
 int validate(const nattn_args* a) {
   if (a == nullptr) return NATTN_EINVAL;
@@ -171,7 +193,15 @@ int validate(const nattn_args* a) {
       (a->sinks && (reinterpret_cast<uintptr_t>(a->sinks) & 3)))
     return NATTN_EALIGN;
   if (a->sinks && a->normalizer != NATTN_SOFTMAX) return NATTN_EUNSUPPORTED;
-  const long long rows = (long long)a->B * a->Hq * a->Tq;
+  if (is_packed(a)) {
+    if (!a->cu_seqlens_k || a->total_q < 1 || a->total_k < 1 || a->Tk < 1) return NATTN_EINVAL;
+    if (is_paged(a)) return NATTN_EINVAL;
+    if (a->weights || a->block_mask) return NATTN_EUNSUPPORTED;
+    if ((long long)a->total_k * a->Hkv >= (1ll << 31)) return NATTN_ETOOLARGE;
+  } else if (a->cu_seqlens_k) {
+    return NATTN_EINVAL;
+  }
+  const long long rows = num_rows(a);
   if (rows >= (1ll << 31) || rows * (long long)(a->d > a->dv ? a->d : a->dv) >= (1ll << 40))
     return NATTN_ETOOLARGE;
   if (is_paged(a)) {
@@ -181,7 +211,7 @@ int validate(const nattn_args* a) {
     if (a->weights || a->block_mask) return NATTN_EUNSUPPORTED;
     if ((long long)a->num_pages * a->Hkv * a->page_size >= (1ll << 31))
       return NATTN_ETOOLARGE;
-  } else {
+  } else if (!is_packed(a)) {
     if ((long long)a->B * a->Hkv * a->Tk >= (1ll << 31)) return NATTN_ETOOLARGE;
     if (a->weights && rows * (long long)a->Tk > kMaxWeights) return NATTN_ETOOLARGE;
   }
@@ -197,11 +227,11 @@ Plan make_plan(const nattn_args* a) {
   Plan pl;
   const bool sparse = a->normalizer == NATTN_SPARSEMAX || a->normalizer == NATTN_ENTMAX15;
   pl.sparse = sparse;
-  const size_t rows = (size_t)a->B * a->Hq * a->Tq;
+  const size_t rows = (size_t)num_rows(a);
   const int group = a->Hq / a->Hkv;
   const bool tc_dims = a->d == a->dv && (a->d == 64 || a->d == 128 || a->d == 256);
+  const bool ps_ok = a->page_size == 32 || a->page_size == 64;
   if (is_paged(a)) {
-    const bool ps_ok = a->page_size == 32 || a->page_size == 64;
     if (tc_dims && ps_ok && group * a->Tq <= 16) {
       pl.path = PATH_DECODE;
       pl.R = group * a->Tq;
@@ -227,7 +257,9 @@ Plan make_plan(const nattn_args* a) {
       pl.total = off;
       return pl;
     }
-  } else if (!a->weights && tc_dims && a->Tk >= 1) {
+  }
+  // dense, packed, and paged chunks too big for the decode kernels: tcgen05
+  if (!a->weights && tc_dims && a->Tk >= 1 && (!is_paged(a) || ps_ok)) {
     pl.path = PATH_TC;
     if (sparse) {
       size_t off = 0;
@@ -297,6 +329,10 @@ Problem to_problem(const nattn_args* a) {
   P.page_size = a->page_size;
   P.bt_stride = a->block_table_stride;
   P.num_pages = a->num_pages;
+  P.cu_q = a->cu_seqlens_q;
+  P.cu_k = a->cu_seqlens_k;
+  P.total_q = a->total_q;
+  P.total_k = a->total_k;
   return P;
 }
 
@@ -323,10 +359,23 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
   constexpr int BN = (D == 256) ? 64 : 128;
   constexpr int KST = 2, VST = 2;
   CUtensorMap mq, mk, mv;
-  if (!make_map_3d(&mq, a->q, D, a->Tq, (long long)a->B * a->Hq, TC_BM) ||
-      !make_map_3d(&mk, a->k, D, a->Tk, (long long)a->B * a->Hkv, BN) ||
-      !make_map_3d(&mv, a->v, D, a->Tk, (long long)a->B * a->Hkv, BN))
-    return NATTN_ECUDA;
+  bool maps;
+  if (is_packed(a)) {
+    maps = make_map_packed(&mq, a->q, D, a->Hq, a->total_q, TC_BM) &&
+           make_map_packed(&mk, a->k, D, a->Hkv, a->total_k, BN) &&
+           make_map_packed(&mv, a->v, D, a->Hkv, a->total_k, BN);
+  } else {
+    maps = make_map_3d(&mq, a->q, D, a->Tq, (long long)a->B * a->Hq, TC_BM);
+    if (is_paged(a)) {  // the pool as rows, one box per page
+      const long long prow = (long long)a->num_pages * a->Hkv * a->page_size;
+      maps = maps && make_map_2d(&mk, a->k, D, prow, a->page_size) &&
+             make_map_2d(&mv, a->v, D, prow, a->page_size);
+    } else {
+      maps = maps && make_map_3d(&mk, a->k, D, a->Tk, (long long)a->B * a->Hkv, BN) &&
+             make_map_3d(&mv, a->v, D, a->Tk, (long long)a->B * a->Hkv, BN);
+    }
+  }
+  if (!maps) return NATTN_ECUDA;
   TcArgs A;
   A.P = P;
   const float log2e = 1.4426950408889634f;
@@ -346,8 +395,19 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
       if ((a->Hq / a->Hkv) % 2 == 0) {
         using PL = PairLayout<D, KST, VST>;
         const bool cap = a->softcap > 0.f || !(A.zscale > 0.f);
-        auto kp = cap ? prefill_pair_kernel<D, KST, VST, true>
-                      : prefill_pair_kernel<D, KST, VST, false>;
+        const bool bm = a->block_mask != nullptr;  // dense mode only
+        decltype(&prefill_pair_kernel<D, KST, VST, true, true, PAIR_DENSE>) kp;
+        if (is_packed(a))
+          kp = cap ? prefill_pair_kernel<D, KST, VST, true, false, PAIR_PACKED>
+                   : prefill_pair_kernel<D, KST, VST, false, false, PAIR_PACKED>;
+        else if (is_paged(a))
+          kp = cap ? prefill_pair_kernel<D, KST, VST, true, false, PAIR_PAGED>
+                   : prefill_pair_kernel<D, KST, VST, false, false, PAIR_PAGED>;
+        else
+          kp = cap ? (bm ? prefill_pair_kernel<D, KST, VST, true, true, PAIR_DENSE>
+                         : prefill_pair_kernel<D, KST, VST, true, false, PAIR_DENSE>)
+                   : (bm ? prefill_pair_kernel<D, KST, VST, false, true, PAIR_DENSE>
+                         : prefill_pair_kernel<D, KST, VST, false, false, PAIR_DENSE>);
         if (allow_smem(kp, PL::ALLOC) != cudaSuccess) return NATTN_ECUDA;
         // persistent: one CTA per SM (shared memory and TMEM allow one), each
         // walking its share of the tiles
@@ -375,6 +435,11 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
   A.sup_list = reinterpret_cast<int2*>(ws + pl.off_supl);
   A.sup_cap = pl.sup_cap;
   if (cudaMemsetAsync(A.ovf_count, 0, sizeof(int), st) != cudaSuccess) return NATTN_ECUDA;
+  // support sizes start at zero: the gather reads every row, and rows that
+  // no sequence owns (packed padding, a sequence rejected on the device) are
+  // never written by the threshold pass
+  if (cudaMemsetAsync(A.sup_count, 0, (size_t)num_rows(a) * sizeof(int), st) != cudaSuccess)
+    return NATTN_ECUDA;
   {
     // d <= 128: each S row split between two warps (eight normalizer warps
     // hide each other's latency; the halves share their bounds); d = 256
@@ -388,7 +453,7 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
   }
   {
     // phase 2: fp32 gather over each row's support list
-    const size_t rows = (size_t)a->B * a->Hq * a->Tq;
+    const size_t rows = (size_t)num_rows(a);
     const unsigned g2 = (unsigned)((rows + GATHER_WARPS - 1) / GATHER_WARPS);
     sparse_gather_kernel<D><<<g2, GATHER_WARPS * 32, 0, st>>>(P, A.sup_count, A.sup_list,
                                                               A.sup_cap, A.tau);
@@ -489,7 +554,7 @@ int run(const nattn_args* a) {
       if (a->d == 128) return launch_decode<128, 64>(a, P, pl, ws, st);
       return launch_decode<256, 64>(a, P, pl, ws, st);
     case PATH_ROWWISE: {
-      const int nrows = a->B * a->Hq * a->Tq;
+      const int nrows = (int)num_rows(a);
       float* slots = pl.row_slots ? reinterpret_cast<float*>(ws + pl.off_slots) : nullptr;
       return launch_rowwise(P, pl, nullptr, nullptr, nrows, slots, pl.row_grid, st);
     }

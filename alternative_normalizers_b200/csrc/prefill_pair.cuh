@@ -63,10 +63,15 @@ struct PairLayout {
 // (one GQA group) of batch b, and the visible key blocks [kb0, kb0 + nblk).
 struct PairTile {
   int b, h0, g, bh0, q0, kb0, kend, nblk;  // nblk: blocks in [kb0, kend) a block mask keeps
+  SeqInfo s;                               // the sequence's lengths / first tokens
 };
 
 // Tile of heaviest-first rank `rank`: under the causal mask the last query
 // tiles see the most keys, so ranks walk the query tiles from the last.
+// Layouts of Q / K / V the kernel is compiled for.
+enum PairLayoutKind { PAIR_DENSE = 0, PAIR_PACKED = 1, PAIR_PAGED = 2 };
+
+template <int LAY>
 __device__ __forceinline__ PairTile pair_tile(const Problem& P, int rank) {
   const int ntq = (P.Tq + TC_BM - 1) / TC_BM;
   const int HP = P.Hq / 2;  // head pairs per batch
@@ -79,11 +84,15 @@ __device__ __forceinline__ PairTile pair_tile(const Problem& P, int rank) {
   T.g = T.h0 / (P.Hq / P.Hkv);
   T.bh0 = T.b * P.Hq + T.h0;
   T.q0 = qt * TC_BM;
-  const int qlast = min(T.q0 + TC_BM - 1, P.Tq - 1);
-  const RowRange r_first = row_range(P, T.q0, P.Tk);
-  const RowRange r_last = row_range(P, qlast, P.Tk);
+  if constexpr (LAY == PAIR_DENSE)
+    T.s = SeqInfo{P.Tq, P.Tk, 0, 0};
+  else
+    T.s = seq_info(P, T.b);
+  const int qlast = min(T.q0 + TC_BM - 1, T.s.Lq - 1);
+  const RowRange r_first = row_range(T.s.Lq, P.causal, P.window, T.q0, T.s.Lk);
+  const RowRange r_last = row_range(T.s.Lq, P.causal, P.window, qlast, T.s.Lk);
   const int klo = max(0, r_first.lo);
-  const int khi = min(P.Tk - 1, r_last.hi);
+  const int khi = (T.q0 < T.s.Lq) ? min(T.s.Lk - 1, r_last.hi) : -1;
   T.kb0 = klo / 128;
   T.kend = (khi >= klo) ? khi / 128 + 1 : T.kb0;
   T.nblk = count_kept<128>(P, T.b, T.h0, T.h0 + 1, qt, T.kb0, T.kend);
@@ -103,25 +112,25 @@ __device__ __forceinline__ int pair_rank(int round, int c, int G) {
 // registers (128 values) for the maximum and the exponentials.
 // `g0` counts the blocks of the CTA's earlier tiles: barrier phases run on
 // across tiles.  Returns false if a wait gave up.
-template <int D, int KST, int VST, bool CAP>
+template <int D, int KST, int VST, bool CAP, bool BM>
 __device__ __forceinline__ bool prefill_pair_normalizer(
     const TcArgs& A, uint8_t* smem, uint32_t tmem, int warp, int lane, int b, int q0, int bh0,
-    int kb0, int kend, int nblk, int g0, uint32_t bar_sf, uint32_t bar_pf, uint32_t bar_pvt,
-    volatile int* abort_flag) {
+    int kb0, int kend, int nblk, const SeqInfo& sq, int g0, uint32_t bar_sf, uint32_t bar_pf,
+    uint32_t bar_pvt, volatile int* abort_flag) {
   using LY = PairLayout<D, KST, VST>;
   constexpr int BN = LY::BN;
   const Problem& P = A.P;
   const int t = warp >> 2, quarter = warp & 3;
   const int row = quarter * 32 + lane;
   const int qi = q0 + row;
-  const bool row_ok = qi < P.Tq;
-  RowRange rr = row_range(P, qi, P.Tk);
+  const bool row_ok = qi < sq.Lq;
+  RowRange rr = row_range(sq.Lq, P.causal, P.window, qi, sq.Lk);
   if (!row_ok) rr = RowRange{1, 0};
-  if (rr.hi > P.Tk - 1) rr.hi = P.Tk - 1;
+  if (rr.hi > sq.Lk - 1) rr.hi = sq.Lk - 1;
   const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
   const uint32_t sbase = lane_base + LY::TM_S + t * BN;
   const uint32_t obase = lane_base + LY::TM_O + t * D;
-  const size_t flat = (size_t)(bh0 + t) * P.Tq + qi;
+  const size_t flat = row_index(P, b, (bh0 + t) % P.Hq, qi, sq);
   // CAP: soft-cap (or a non-positive scale), scores go through tc_z; else
   // max(z) = scale * max(s) and exp2(z - m) is one FFMA + EX2 per score
   constexpr bool fast = !CAP;
@@ -135,7 +144,7 @@ __device__ __forceinline__ bool prefill_pair_normalizer(
   // block mask: the pair walks the blocks either head keeps; a block this
   // tile's head drops is masked whole
   const int qb = q0 >> 7, hp = bh0 % P.Hq, hown = hp + t;
-  int kb = next_kept<BN>(P, b, hp, hp + 1, qb, kb0, kend);
+  int kb = BM ? next_kept<BN>(P, b, hp, hp + 1, qb, kb0, kend) : kb0;
   int nvis = 0;  // visible keys in kept blocks (row_nnz)
 
   for (int j = 0; j < nblk; ++j) {
@@ -145,17 +154,17 @@ __device__ __forceinline__ bool prefill_pair_normalizer(
     }
     tc_fence_after();
     const int jb = kb * BN;
-    const bool own = block_kept(P, b, hown, qb, kb);
+    const bool own = !BM || block_kept(P, b, hown, qb, kb);
     const bool edge = !own || !(rr.lo <= jb && rr.hi >= jb + BN - 1);
     int kl = rr.lo - jb;
     unsigned span = (unsigned)(rr.hi - rr.lo);
     if (rr.hi < rr.lo || !own) {
       kl = BN;
       span = 0;
-    } else {
+    } else if (BM) {
       nvis += max(0, min(rr.hi, jb + BN - 1) - max(rr.lo, jb) + 1);
     }
-    kb = next_kept<BN>(P, b, hp, hp + 1, qb, kb + 1, kend);
+    kb = BM ? next_kept<BN>(P, b, hp, hp + 1, qb, kb + 1, kend) : kb + 1;
     // the whole S row (128 scores) in registers: one TMEM read per block;
     // x is the raw score on the fast path, else z in log2 units; masked
     // entries -inf
@@ -247,11 +256,14 @@ __device__ __forceinline__ bool prefill_pair_normalizer(
   }
   if (row_ok && P.row_stat) P.row_stat[flat] = stat;
   if (row_ok && P.row_nnz)
-    P.row_nnz[flat] = P.block_mask ? nvis : (rr.hi >= rr.lo ? rr.hi - rr.lo + 1 : 0);
+    P.row_nnz[flat] = BM ? nvis : (rr.hi >= rr.lo ? rr.hi - rr.lo + 1 : 0);
   return alive;
 }
 
-template <int D, int KST, int VST, bool CAP>
+// BM: a block mask is given; LAY: dense, packed or paged Q / K / V (separate
+// instances, so that the dense launches without a block mask carry none of
+// the other cases' per-block work)
+template <int D, int KST, int VST, bool CAP, bool BM, int LAY>
 __global__ void __launch_bounds__(PAIR_THREADS, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq,
                         const __grid_constant__ CUtensorMap tmk,
@@ -318,9 +330,9 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
     for (int round = 0;; ++round) {
       const int rank = pair_rank(round, cta, G);
       if (rank >= ntiles) break;
-      const PairTile T = pair_tile(P, rank);
-      if (!prefill_pair_normalizer<D, KST, VST, CAP>(A, smem, tmem, warp, lane, T.b, T.q0,
-                                                      T.bh0, T.kb0, T.kend, T.nblk, g0,
+      const PairTile T = pair_tile<LAY>(P, rank);
+      if (!prefill_pair_normalizer<D, KST, VST, CAP, BM>(A, smem, tmem, warp, lane, T.b, T.q0,
+                                                      T.bh0, T.kb0, T.kend, T.nblk, T.s, g0,
                                                       bar_sfull(warp >> 2),
                                                       bar_pfull(warp >> 2), bar_pv(warp >> 2),
                                                       abort_flag))
@@ -334,12 +346,13 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
       tma_prefetch_desc(&tmq);
       tma_prefetch_desc(&tmk);
       tma_prefetch_desc(&tmv);
+      constexpr bool packed = LAY == PAIR_PACKED;
       int g0 = 0, tq = 0;  // blocks and tiles (with blocks) already loaded
       bool ok = true;
       for (int round = 0; ok; ++round) {
         const int rank = pair_rank(round, cta, G);
         if (rank >= ntiles) break;
-        const PairTile T = pair_tile(P, rank);
+        const PairTile T = pair_tile<LAY>(P, rank);
         if (T.nblk == 0) continue;
         // the previous tile's QK products have read its Q tiles
         if (tq > 0 && !mbar_wait(bar_qempty, (tq - 1) & 1, abort_flag)) break;
@@ -348,8 +361,9 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
         for (int t = 0; t < 2; ++t)
 #pragma unroll
           for (int x = 0; x < D / 64; ++x)
-            tma_load_3d(smem_addr(smem + LY::OFF_Q + t * LY::QBYTES + x * TC_BM * 128), &tmq,
-                        bar_q, x * 64, T.q0, T.bh0 + t);
+            tma_load_rows(smem_addr(smem + LY::OFF_Q + t * LY::QBYTES + x * TC_BM * 128), &tmq,
+                          bar_q, x * 64, packed ? T.s.q0 + T.q0 : T.q0,
+                          packed ? T.h0 + t : T.bh0 + t, packed);
         int kb = next_kept<BN>(P, T.b, T.h0, T.h0 + 1, T.q0 >> 7, T.kb0, T.kend);
         for (int j = 0; j < T.nblk; ++j, kb = next_kept<BN>(P, T.b, T.h0, T.h0 + 1, T.q0 >> 7,
                                                             kb + 1, T.kend)) {
@@ -361,10 +375,14 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
           }
           mbar_expect_tx(bar_kfull(ks), LY::KBYTES);
           uint8_t* kdst = smem + LY::OFF_K + ks * LY::KBYTES;
+          if constexpr (LAY == PAIR_DENSE) {
 #pragma unroll
-          for (int x = 0; x < D / 64; ++x)
-            tma_load_3d(smem_addr(kdst + x * BN * 128), &tmk, bar_kfull(ks), x * 64, kb * BN,
-                        T.b * P.Hkv + T.g);
+            for (int x = 0; x < D / 64; ++x)
+              tma_load_3d(smem_addr(kdst + x * BN * 128), &tmk, bar_kfull(ks), x * 64, kb * BN,
+                          T.b * P.Hkv + T.g);
+          } else {
+            tma_load_kv<D, BN>(P, &tmk, kdst, bar_kfull(ks), T.b, T.g, kb, T.s);
+          }
           const int vs = gj % VST;
           if (gj >= VST && !mbar_wait(bar_vempty(vs), ((gj / VST) + 1) & 1, abort_flag)) {
             ok = false;
@@ -372,10 +390,14 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
           }
           mbar_expect_tx(bar_vfull(vs), LY::VBYTES);
           uint8_t* vdst = smem + LY::OFF_V + vs * LY::VBYTES;
+          if constexpr (LAY == PAIR_DENSE) {
 #pragma unroll
-          for (int x = 0; x < D / 64; ++x)
-            tma_load_3d(smem_addr(vdst + x * BN * 128), &tmv, bar_vfull(vs), x * 64, kb * BN,
-                        T.b * P.Hkv + T.g);
+            for (int x = 0; x < D / 64; ++x)
+              tma_load_3d(smem_addr(vdst + x * BN * 128), &tmv, bar_vfull(vs), x * 64, kb * BN,
+                          T.b * P.Hkv + T.g);
+          } else {
+            tma_load_kv<D, BN>(P, &tmv, vdst, bar_vfull(vs), T.b, T.g, kb, T.s);
+          }
         }
         g0 += T.nblk;
         ++tq;
@@ -401,7 +423,7 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
       for (int round = 0; ok; ++round) {
         const int rank = pair_rank(round, cta, G);
         if (rank >= ntiles) break;
-        const PairTile T = pair_tile(P, rank);
+        const PairTile T = pair_tile<LAY>(P, rank);
         const int nblk = T.nblk;
         if (nblk == 0) continue;
         ok = mbar_wait_spin(bar_q, tq & 1, abort_flag);

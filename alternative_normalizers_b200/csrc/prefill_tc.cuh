@@ -61,9 +61,69 @@ struct TcArgs {
   int* ovf_rows;     // TAU: rows whose candidate buffer overflowed
   int* ovf_count;    // TAU: number of such rows (zeroed before the launch)
   int* sup_count;    // TAU: support size of every row (0 for overflowed rows)
-  int2* sup_list;    // TAU: [rows][sup_cap] (key index, weight bits)
+  int2* sup_list;    // TAU: [rows][sup_cap] (value row of the key, weight bits)
   int sup_cap;
 };
+
+// Rows [row0, row0 + box) of head plane `plane` (batch * heads + head for the
+// dense layout, the head for the packed one) of a Q / K / V tensor, 64
+// columns from column x: dense tensor maps are [planes][rows][64-wide],
+// packed ones [rows][planes][64-wide] (FlashAttention-style [total, H, d]).
+__device__ __forceinline__ void tma_load_rows(uint32_t dst, const void* map, uint32_t bar, int x,
+                                              int row0, int plane, bool packed) {
+  if (packed)
+    tma_load_3d(dst, map, bar, x, plane, row0);
+  else
+    tma_load_3d(dst, map, bar, x, row0, plane);
+}
+
+// Key (or value) block kb (keys [kb * BN, kb * BN + BN)) of sequence b, kv
+// head g into a 128-byte-swizzled tile of DIM / 64 boxes of BN rows.  Paged
+// mode: the map views the pool as rows [num_pages * Hkv * page_size][DIM]
+// with one box per page; pages past the sequence's end load page 0 (their
+// keys are masked), an out-of-range page id records NATTN_EBOUNDS and loads
+// page 0 too ("HF Attention Normalizers", section "Differentiable Paged
+// Attention": the kernel reads physical pages through the block table).
+template <int DIM, int BN>
+__device__ __forceinline__ void tma_load_kv(const Problem& P, const CUtensorMap* map, uint8_t* dst,
+                                            uint32_t bar, int b, int g, int kb, const SeqInfo& s) {
+  if (P.block_table != nullptr) {
+    const int ps = P.page_size;
+    for (int p = 0; p < BN / ps; ++p) {
+      const int lp = (kb * BN) / ps + p;
+      int page = 0;
+      if (lp * ps < s.Lk) {
+        page = P.block_table[(size_t)b * P.bt_stride + lp];
+        if (page < 0 || page >= P.num_pages) {
+          set_status(NATTN_EBOUNDS);
+          page = 0;
+        }
+      }
+#pragma unroll
+      for (int x = 0; x < DIM / 64; ++x)
+        tma_load_2d(smem_addr(dst + x * BN * 128 + p * ps * 128), map, bar, x * 64,
+                    (page * P.Hkv + g) * ps);
+    }
+    return;
+  }
+  const bool packed = P.cu_q != nullptr;
+#pragma unroll
+  for (int x = 0; x < DIM / 64; ++x)
+    tma_load_rows(smem_addr(dst + x * BN * 128), map, bar, x * 64,
+                  packed ? s.k0 + kb * BN : kb * BN, packed ? g : b * P.Hkv + g, packed);
+}
+
+// Row of value row j of sequence b, kv head g in the V tensor viewed as rows
+// of dv elements (the sparse gather's address of a support key).
+__device__ __forceinline__ int value_row(const Problem& P, int b, int g, int j, const SeqInfo& s) {
+  if (P.cu_q != nullptr) return (s.k0 + j) * P.Hkv + g;
+  if (P.block_table != nullptr) {
+    int page = P.block_table[(size_t)b * P.bt_stride + j / P.page_size];
+    if (page < 0 || page >= P.num_pages) page = 0;  // recorded by the loads
+    return (page * P.Hkv + g) * P.page_size + j % P.page_size;
+  }
+  return (b * P.Hkv + g) * P.Tk + j;
+}
 
 // NH = 2 splits every S row between two warps (columns [0, BN/2) and
 // [BN/2, BN)).  In the online mode each half keeps its own running maximum,
@@ -220,11 +280,14 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
   const int b = bh / P.Hq, h = bh % P.Hq;
   const int g = h / (P.Hq / P.Hkv);
   const int q0 = qt * TC_BM;
-  const int qlast = min(q0 + TC_BM - 1, P.Tq - 1);
-  const RowRange r_first = row_range(P, q0, P.Tk);
-  const RowRange r_last = row_range(P, qlast, P.Tk);
+  // this sequence's lengths (packed and paged modes have their own)
+  const SeqInfo sq = seq_info(P, b);
+  const bool packed = P.cu_q != nullptr;
+  const int qlast = min(q0 + TC_BM - 1, sq.Lq - 1);
+  const RowRange r_first = row_range(sq.Lq, P.causal, P.window, q0, sq.Lk);
+  const RowRange r_last = row_range(sq.Lq, P.causal, P.window, qlast, sq.Lk);
   const int klo = max(0, r_first.lo);
-  const int khi = min(P.Tk - 1, r_last.hi);
+  const int khi = (q0 < sq.Lq) ? min(sq.Lk - 1, r_last.hi) : -1;
   const int kb0 = klo / BN;
   const int kend = (khi >= klo) ? khi / BN + 1 : kb0;
   // blocks of [kb0, kend) the block mask keeps (all of them without one)
@@ -282,28 +345,22 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
       mbar_expect_tx(bar_q, LY::QBYTES);
 #pragma unroll
       for (int x = 0; x < D / 64; ++x)
-        tma_load_3d(smem_addr(smem + LY::OFF_Q + x * TC_BM * 128), &tmq, bar_q, x * 64, q0,
-                    bh);
+        tma_load_rows(smem_addr(smem + LY::OFF_Q + x * TC_BM * 128), &tmq, bar_q, x * 64,
+                      packed ? sq.q0 + q0 : q0, packed ? h : bh, packed);
       int kb = next_kept<BN>(P, b, h, h, qt, kb0, kend);
       for (int j = 0; j < nblk; ++j, kb = next_kept<BN>(P, b, h, h, qt, kb + 1, kend)) {
         const int ks = j % KST;
         if (j >= KST && !mbar_wait(bar_kempty(ks), ((j / KST) + 1) & 1, abort_flag)) break;
         mbar_expect_tx(bar_kfull(ks), LY::KBYTES);
-        uint8_t* kdst = smem + LY::OFF_K + ks * LY::KBYTES;
-#pragma unroll
-        for (int x = 0; x < D / 64; ++x)
-          tma_load_3d(smem_addr(kdst + x * BN * 128), &tmk, bar_kfull(ks), x * 64, kb * BN,
-                      b * P.Hkv + g);
+        tma_load_kv<D, BN>(P, &tmk, smem + LY::OFF_K + ks * LY::KBYTES, bar_kfull(ks), b, g, kb,
+                           sq);
         if constexpr (MODE != TC_TAU) {
           const int vs = j % VST;
           if (j >= VST && !mbar_wait(bar_vempty(vs), ((j / VST) + 1) & 1, abort_flag))
             break;
           mbar_expect_tx(bar_vfull(vs), LY::VBYTES);
-          uint8_t* vdst = smem + LY::OFF_V + vs * LY::VBYTES;
-#pragma unroll
-          for (int x = 0; x < DV / 64; ++x)
-            tma_load_3d(smem_addr(vdst + x * BN * 128), &tmv, bar_vfull(vs), x * 64,
-                        kb * BN, b * P.Hkv + g);
+          tma_load_kv<DV, BN>(P, &tmv, smem + LY::OFF_V + vs * LY::VBYTES, bar_vfull(vs), b, g,
+                              kb, sq);
         }
       }
     }
@@ -377,12 +434,12 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
     const int cbase = half * NC;
     const int row = quarter * 32 + lane;
     const int qi = q0 + row;
-    const bool row_ok = qi < P.Tq;
-    RowRange rr = row_range(P, qi, P.Tk);
+    const bool row_ok = qi < sq.Lq;
+    RowRange rr = row_range(sq.Lq, P.causal, P.window, qi, sq.Lk);
     if (!row_ok) rr = RowRange{1, 0};
-    if (rr.hi > P.Tk - 1) rr.hi = P.Tk - 1;
+    if (rr.hi > sq.Lk - 1) rr.hi = sq.Lk - 1;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const size_t flat = ((size_t)bh * P.Tq + qi);
+    const size_t flat = row_index(P, b, h, qi, sq);
     // fast path: no soft-cap and a positive scale, so max(z) = scale * max(s)
     // and exp2(z - m) is one FFMA + EX2 per score
     const bool fast = !(P.softcap > 0.f) && A.zscale > 0.f;
@@ -477,21 +534,24 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
         const float msafe = (m_use == -INFINITY) ? 0.f : m_use;
         const float fa = fast ? zs : 1.f;  // p = exp2(x * fa - msafe)
         float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-        for (int c = 0; c < LDC / 64; ++c) {  // 64 scores -> 32 packed columns
-          uint32_t pk[32];
-          exp2_pack64(&r[c * 64], fa, msafe, s0, s1, pk);
-          tmem_st32(paddr + c * 32, pk);
+        static_assert(LDC == 64, "one 64-score chunk per online step");
+        uint32_t pk[32];  // 64 scores -> 32 packed columns
+        exp2_pack64(&r[0], fa, msafe, s0, s1, pk);
+        // P(j) is stored only once the previous block's PV has completed, so
+        // no TMEM store overlaps a product that reads TMEM (that product was
+        // issued a whole block of exponentials earlier: the wait rarely
+        // stalls); this also orders the O rescale below
+        if (j > 0 &&
+            !__all_sync(0xffffffffu, mbar_wait_spin(bar_pv, (j - 1) & 1, abort_flag))) {
+          alive = false;
+          break;
         }
+        tc_fence_after();
+        tmem_st32(paddr, pk);
         tmem_st_wait();
         l_run = l_run * alpha + (s0 + s1);
         // rescale O when the maximum moved (warp-uniform TMEM access)
         if (__any_sync(0xffffffffu, resc) && j > 0) {
-          if (!__all_sync(0xffffffffu, mbar_wait(bar_pv, (j - 1) & 1, abort_flag))) {
-            alive = false;
-            break;
-          }
-          tc_fence_after();
           const uint32_t oaddr = lane_base + LY::TM_O + half * DV;
 #pragma unroll 1
           for (int c = 0; c < DV / 32; ++c) {
@@ -673,7 +733,10 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
             for (int i = 0; i < n; ++i) {
               const int2 e = src[i];
               const float x = __int_as_float(e.y) * vs - t;
-              if (x > 0.f) dst[nsup++] = make_int2(e.x, __float_as_int(entmax ? x * x : x));
+              // the gather reads the support key's value row by its row index
+              if (x > 0.f)
+                dst[nsup++] =
+                    make_int2(value_row(P, b, g, e.x, sq), __float_as_int(entmax ? x * x : x));
             }
           };
           emit(b0, n0);
@@ -773,7 +836,8 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
 
 
 // Sparse phase 2 (default): O = sum over the row's support of p_j V_j, in
-// fp32 on CUDA cores, from the (key, weight) list the threshold pass wrote.
+// fp32 on CUDA cores, from the (value row, weight) list the threshold pass
+// wrote.
 // The support of sparsemax / 1.5-entmax is a handful of keys per row, so
 // this touches |support| value rows instead of multiplying every block, and
 // the weights enter the sum in full precision.  One warp per query row; lane
@@ -787,18 +851,19 @@ __global__ void __launch_bounds__(GATHER_WARPS * 32)
                          const float* __restrict__ tau) {
   constexpr int PER = DV / 32;  // columns per lane (2, 4 or 8)
   const int lane = threadIdx.x & 31;
-  const size_t rows = (size_t)P.B * P.Hq * P.Tq;
+  const size_t rows =
+      P.cu_q != nullptr ? (size_t)P.total_q * P.Hq : (size_t)P.B * P.Hq * P.Tq;
   const size_t flat = (size_t)blockIdx.x * GATHER_WARPS + (threadIdx.x >> 5);
   if (flat >= rows) return;
-  const int h = (int)((flat / P.Tq) % P.Hq);
-  const int b = (int)(flat / ((size_t)P.Tq * P.Hq));
-  const int g = h / (P.Hq / P.Hkv);
-  const int n = sup_count[flat];
+  // packed: rows past the last sequence belong to no sequence
+  if (P.cu_q != nullptr && flat >= (size_t)min(P.cu_q[P.B], P.total_q) * P.Hq) return;
+  const int n = min(sup_count[flat], sup_cap);
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
   if (n > 0) {
-    const bf16* vbase = P.v + ((size_t)b * P.Hkv + g) * (size_t)P.Tk * DV + lane * PER;
+    // support entries carry the value row of each key (see value_row)
+    const bf16* vbase = P.v + lane * PER;
     const int2* lst = sup_list + flat * (size_t)sup_cap;
     for (int e0 = 0; e0 < n; e0 += 32) {
       const int2 mine = (e0 + lane < n) ? lst[e0 + lane] : make_int2(0, 0);

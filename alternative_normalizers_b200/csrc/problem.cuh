@@ -32,7 +32,52 @@ struct Problem {
   const int32_t* block_table;
   const int32_t* seqlens;
   int page_size, bt_stride, num_pages;
+  // packed variable-length mode (cu_q != nullptr): q [total_q, Hq, d],
+  // k / v [total_k, Hkv, d | dv], out [total_q, Hq, dv], row_stat and
+  // row_nnz [total_q, Hq]; sequence b owns query tokens [cu_q[b], cu_q[b+1])
+  // and key tokens [cu_k[b], cu_k[b+1]); Tq / Tk are the largest lengths
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int total_q, total_k;
 };
+
+// One sequence's lengths and, in packed mode, its first query / key token.
+// Lengths outside the declared bounds are recorded as NATTN_EBOUNDS and the
+// sequence is treated as empty.
+struct SeqInfo {
+  int Lq, Lk, q0, k0;
+};
+
+__device__ __forceinline__ SeqInfo seq_info(const Problem& P, int b) {
+  SeqInfo s{P.Tq, P.Tk, 0, 0};
+  if (P.cu_q != nullptr) {
+    s.q0 = P.cu_q[b];
+    s.k0 = P.cu_k[b];
+    s.Lq = P.cu_q[b + 1] - s.q0;
+    s.Lk = P.cu_k[b + 1] - s.k0;
+    if (s.q0 < 0 || s.k0 < 0 || s.Lq < 0 || s.Lk < 0 || s.Lq > P.Tq || s.Lk > P.Tk ||
+        s.q0 + s.Lq > P.total_q || s.k0 + s.Lk > P.total_k) {
+      set_status(NATTN_EBOUNDS);
+      s.Lq = s.Lk = 0;
+      s.q0 = s.k0 = 0;
+    }
+  } else if (P.block_table != nullptr) {
+    s.Lk = P.seqlens[b];
+    if (s.Lk < 0 || s.Lk > P.Tk || s.Lk > P.bt_stride * P.page_size) {
+      set_status(NATTN_EBOUNDS);
+      s.Lk = 0;
+    }
+  }
+  return s;
+}
+
+// Flat index of query row i of head h of sequence b: the row of out,
+// row_stat and row_nnz (and of every per-row scratch array).
+__device__ __forceinline__ size_t row_index(const Problem& P, int b, int h, int i,
+                                            const SeqInfo& s) {
+  return P.cu_q != nullptr ? (size_t)(s.q0 + i) * P.Hq + h
+                           : ((size_t)b * P.Hq + h) * P.Tq + i;
+}
 
 // Inclusive key range [lo, hi] visible to query row i when the row's key
 // length is L.  The query sits at key position pos = i + L - Tq (causal
@@ -107,10 +152,12 @@ __device__ __forceinline__ int count_kept(const Problem& P, int b, int h0, int h
 }
 
 // Address of key (or value) row j of sequence b, kv head g.  Dense layout
-// [B, Hkv, Tk, dim]; paged pool [num_pages, Hkv, page_size, dim] through the
-// block table.  An out-of-range page id sets `bad` and returns nullptr.
+// [B, Hkv, Tk, dim]; packed layout [total_k, Hkv, dim]; paged pool
+// [num_pages, Hkv, page_size, dim] through the block table.  An
+// out-of-range page id sets `bad` and returns nullptr.
 __device__ __forceinline__ const bf16* key_row(const Problem& P, const bf16* base, int dim,
                                                int b, int g, int j, bool& bad) {
+  if (P.cu_q != nullptr) return base + ((size_t)(P.cu_k[b] + j) * P.Hkv + g) * dim;
   if (P.block_table == nullptr)
     return base + (((size_t)b * P.Hkv + g) * P.Tk + j) * dim;
   const int page = P.block_table[(size_t)b * P.bt_stride + j / P.page_size];

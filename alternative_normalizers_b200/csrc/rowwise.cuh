@@ -139,17 +139,27 @@ __global__ void __launch_bounds__(ROW_THREADS)
 
   for (int r = blockIdx.x; r < nrows; r += gridDim.x) {
     const int flat = row_list ? row_list[r] : r;
-    const int i = flat % P.Tq;
-    const int h = (flat / P.Tq) % P.Hq;
-    const int b = flat / (P.Tq * P.Hq);
-    const int g = h / group;
-    int L = P.Tk;
-    bool bad = false;
-    if (P.block_table) {
-      L = P.seqlens[b];
-      if (L < 0 || L > P.Tk || L > P.bt_stride * P.page_size) bad = true;
+    int b, h, i;
+    if (P.cu_q != nullptr) {
+      // packed rows are [total_q][Hq]: the token's sequence by binary search
+      const int tok = flat / P.Hq;
+      h = flat % P.Hq;
+      int lo = 0, hi = P.B - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (P.cu_q[mid] <= tok) lo = mid; else hi = mid - 1;
+      }
+      b = lo;
+      i = tok - P.cu_q[b];
+    } else {
+      i = flat % P.Tq;
+      h = (flat / P.Tq) % P.Hq;
+      b = flat / (P.Tq * P.Hq);
     }
-    const RowRange rr = row_range(P, i, bad ? 0 : L);
+    const int g = h / group;
+    bool bad = false;
+    const SeqInfo sq = seq_info(P, b);  // out-of-range lengths: an empty row
+    const RowRange rr = row_range(sq.Lq, P.causal, P.window, i, sq.Lk);
     int n = rr.hi - rr.lo + 1;
     if (n < 0) n = 0;
     float* sc = sc_smem;

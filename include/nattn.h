@@ -128,6 +128,32 @@ enum {
  *            the special case sinks[h] = 0.  Any other normalizer with sinks:
  *            NATTN_EUNSUPPORTED.  4-byte aligned (NATTN_EALIGN).
  *
+ * Packed variable-length mode (cu_seqlens_q != NULL; "HF Attention
+ * Normalizers", section "Packed Variable-Length Attention": FlashAttention-
+ * style packed layouts with cumulative sequence lengths, GQA, different
+ * query and key lengths, per-request bottom-right causal alignment, one grid
+ * over the packed batch with no padded staging):
+ *   q        bf16 [total_q, Hq, d]
+ *   k        bf16 [total_k, Hkv, d]
+ *   v        bf16 [total_k, Hkv, dv]
+ *   out      bf16 [total_q, Hq, dv]; row_stat, row_nnz [total_q, Hq]
+ *   cu_seqlens_q, cu_seqlens_k  int32 [B + 1], device memory, nondecreasing
+ *            from 0: sequence b owns query tokens [cu_seqlens_q[b],
+ *            cu_seqlens_q[b+1]) and key tokens [cu_seqlens_k[b],
+ *            cu_seqlens_k[b+1]); its query row i sits at key position
+ *            i + Lk_b - Lq_b.
+ *   Tq, Tk   the largest query and key length of any sequence (they size the
+ *            grid; a longer sequence is recorded as NATTN_EBOUNDS on the
+ *            device and computed as empty).
+ *   total_q, total_k  rows of q and of k / v (>= the last cumulative length).
+ * Not with a block table, dense weights or a block mask
+ * (NATTN_EUNSUPPORTED).
+ *
+ * Paged prefill: in paged mode a chunk of Tq new tokens per sequence against
+ * a page pool with 32- or 64-token pages runs on the same tensor-core
+ * kernels as dense prefill whenever (Hq / Hkv) * Tq > 16 (fewer rows per
+ * key/value head go to the split-KV decode kernels).
+ *
  * Block mask ("Attention variants: what to open up, and how far",
  * TensorCAD, section "C. Keep the fused kernel": a mask yields a block mask,
  * and whole blocks that are masked out are skipped):
@@ -172,6 +198,10 @@ typedef struct nattn_args {
                                below); NATTN_SOFTMAX only                   */
   const uint8_t* block_mask;/* 128 x 128 block mask, or NULL (see below);
                                dense mode only                              */
+  const int32_t* cu_seqlens_q; /* packed variable-length mode (see below),  */
+  const int32_t* cu_seqlens_k; /* or NULL                                   */
+  int total_q;              /* packed mode: rows of q / out                 */
+  int total_k;              /* packed mode: rows of k / v                   */
 } nattn_args;
 
 /*
