@@ -613,6 +613,90 @@ class BwdRunner:
         return 2.5 * self.w.useful_flops()
 
 
+class ArgsRunner:
+    """Timing target for prebuilt argument blocks: one nattn_fwd_ex per call."""
+
+    def __init__(self, name, normalizers, args, keep, units):
+        from types import SimpleNamespace
+        from alternative_normalizers_b200 import binding
+        self.w = SimpleNamespace(name=name, normalizers=tuple(normalizers))
+        self.binding, self.args, self.keep, self._units = binding, args, keep, units
+
+    def call(self, n):
+        rc = self.binding.nattn_fwd_ex(self.args[n])
+        if rc != 0:
+            raise RuntimeError(f"nattn_fwd_ex({n}) failed: {rc}")
+
+    def units(self):
+        return self._units
+
+
+def varlen_runner(dev):
+    """The headline layer's heads (Hq=32, Hkv=8, d=128, causal) over one
+    packed batch of four requests of 4096, 2048, 1536 and 512 tokens
+    ([total, H, d] layouts, cumulative lengths)."""
+    import torch
+    from alternative_normalizers_b200 import binding
+    lens = [4096, 2048, 1536, 512]
+    tot, Hq, Hkv, d = sum(lens), 32, 8, 128
+    g = torch.Generator().manual_seed(2024)
+    mk = lambda *sh: torch.randn(*sh, generator=g).to(torch.bfloat16).to(dev)
+    q, k, v = mk(tot, Hq, d), mk(tot, Hkv, d), mk(tot, Hkv, d)
+    cu = torch.tensor([0] + list(__import__("itertools").accumulate(lens)),
+                      dtype=torch.int32, device=dev)
+    out = torch.empty(tot, Hq, d, dtype=torch.bfloat16, device=dev)
+    st = torch.empty(tot, Hq, dtype=torch.float32, device=dev)
+    args, keep = {}, [q, k, v, cu, out, st]
+    for n in ("softmax", "sparsemax"):
+        a = binding.NattnArgs()
+        a.q, a.k, a.v, a.out, a.row_stat = (t.data_ptr() for t in (q, k, v, out, st))
+        a.B, a.Hq, a.Hkv, a.d, a.dv, a.Tq, a.Tk = len(lens), Hq, Hkv, d, d, max(lens), max(lens)
+        a.scale, a.normalizer, a.causal = d ** -0.5, binding.NORMALIZER_IDS[n], 1
+        a.cu_seqlens_q = a.cu_seqlens_k = cu.data_ptr()
+        a.total_q = a.total_k = tot
+        a.stream = torch.cuda.current_stream(dev).cuda_stream
+        need = binding.nattn_workspace_size(a)
+        if need:
+            ws = torch.empty(need, dtype=torch.uint8, device=dev)
+            keep.append(ws)
+            a.workspace, a.workspace_bytes = ws.data_ptr(), need
+        args[n] = a
+    pairs = sum(L * (L + 1) // 2 for L in lens)
+    return ArgsRunner("packed_varlen", args.keys(), args, keep, 4.0 * d * pairs * Hq)
+
+
+def paged_prefill_runner(dev):
+    """Chunked prefill into a paged cache: 8 requests, each with 1024 new
+    query tokens after 3072 cached ones (4096 keys), Hq=32, Hkv=8, d=128,
+    64-token pages in a random permutation of the pool, causal."""
+    import torch
+    from alternative_normalizers_b200 import binding
+    B, Tq, L, Hq, Hkv, d, ps = 8, 1024, 4096, 32, 8, 128, 64
+    g = torch.Generator().manual_seed(2025)
+    mk = lambda *sh: torch.randn(*sh, generator=g).to(torch.bfloat16).to(dev)
+    npg = L // ps
+    q = mk(B, Hq, Tq, d)
+    kp, vp = mk(B * npg, Hkv, ps, d), mk(B * npg, Hkv, ps, d)
+    table = torch.randperm(B * npg, generator=g).to(torch.int32).view(B, npg).to(dev)
+    lens = torch.full((B,), L, dtype=torch.int32, device=dev)
+    out = torch.empty(B, Hq, Tq, d, dtype=torch.bfloat16, device=dev)
+    st = torch.empty(B, Hq, Tq, dtype=torch.float32, device=dev)
+    args, keep = {}, [q, kp, vp, table, lens, out, st]
+    for n in ("softmax", "sparsemax"):
+        a = binding.build_args(q, kp, vp, out, st, None, normalizer=n, causal=True,
+                               scale=d ** -0.5, block_table=table, seqlens=lens,
+                               page_size=ps, max_seqlen=L)
+        need = binding.nattn_workspace_size(a)
+        if need:
+            ws = torch.empty(need, dtype=torch.uint8, device=dev)
+            keep.append(ws)
+            a.workspace, a.workspace_bytes = ws.data_ptr(), need
+        args[n] = a
+    # query i of a request sits at key position i + 3072: sees 3073 + i keys
+    pairs = Tq * (L - Tq) + Tq * (Tq + 1) // 2
+    return ArgsRunner("paged_prefill", args.keys(), args, keep, 4.0 * d * pairs * B * Hq)
+
+
 def detail(args, dev, flush):
     """The other workload shapes, each normalizer timed like the headline."""
     import torch
@@ -724,6 +808,22 @@ def detail(args, dev, flush):
         torch.cuda.empty_cache()
     except Exception as exc:
         res["qwen3_8b_prefill_doc_mask"] = {"error": repr(exc)[:200]}
+    # packed variable-length batch and chunked paged prefill (exact pairs)
+    for make in (varlen_runner, paged_prefill_runner):
+        try:
+            r = make(dev)
+            per = time_runner(r, max(3, args.steps // 2), 2, flush)
+            vals = {n: round(r.units() / (t * 1e-3) / 1e12, 1) for n, t in per.items()}
+            res[r.w.name] = {
+                "unit": "useful TFLOP/s (exact allowed pairs)", "value": vals,
+                "ms": {n: round(t, 4) for n, t in per.items()},
+                "roofline_frac": {n: round(v / peaks["bf16_tflops"], 4)
+                                  for n, v in vals.items()},
+                "roofline_denominator": "of measured bf16_tflops (burst)"}
+            del r
+            torch.cuda.empty_cache()
+        except Exception as exc:
+            res[make.__name__] = {"error": repr(exc)[:200]}
     return res
 
 
