@@ -26,14 +26,19 @@
 //           m0 = 0, l0 = 1.  The running maximum is only moved (and O
 //           rescaled) when it grows by more than 2^8, which keeps rescaling
 //           off the common path.
-//   TAU     sparse phase 1: S only.  Each row streams its scores once and
-//           keeps a small buffer of the only entries that can still be in the
-//           support (those above a running lower bound of tau); the exact
-//           threshold is solved on that buffer at the end ("HF Attention
-//           Normalizers", section "Important Limitations": the sparse kernels
-//           stream K/V tiles, solve the global normalization threshold and
-//           save one threshold per query row).  Rows whose candidates
-//           overflow the buffer are listed for the row-wise kernel.
+//   TAU     sparse phase 1: S only, in two passes over the key blocks.  The
+//           bound pass keeps 32 bucket maxima per thread (two three-input
+//           max operations per four scores, no branches) and solves the
+//           exact threshold of those distinct keys: a lower bound of the
+//           row's.  The candidate pass keeps every key above that fixed
+//           bound in a small buffer, and the exact threshold is solved on the
+//           buffer at the end ("HF Attention Normalizers", section "Important
+//           Limitations": the sparse kernels stream K/V tiles, solve the
+//           global normalization threshold and save one threshold per query
+//           row).  The second QK product is cheap next to per-score work on
+//           the CUDA cores, which sets this mode's speed.  Rows whose
+//           candidates overflow the buffer are listed for the row-wise
+//           kernel.
 // Sparse phase 2 is sparse_gather_kernel below: an fp32 sum over each row's
 // support list.
 #pragma once
@@ -47,10 +52,12 @@ enum TcMode { TC_ONLINE = 0, TC_TAU = 1 };
 
 constexpr int TC_THREADS = 192;
 constexpr int TC_BM = 128;
-// candidate buffer entries per row in the threshold pass (value + key index)
+// candidate buffer entries per row in the threshold pass (value + key index);
+// with the bound pass's bound the candidates of a row are its support and a
+// few keys more
 template <int D>
 struct TauCap {
-  static constexpr int value = (D >= 256) ? 88 : 112;
+  static constexpr int value = (D >= 256) ? 72 : 92;
 };
 
 struct TcArgs {
@@ -135,7 +142,17 @@ __device__ __forceinline__ int value_row(const Problem& P, int b, int g, int j, 
 template <int D, int DV, int BN, int KST, int VST, int MODE, int NH = 1>
 struct TcLayout {
   static constexpr int NWN = 4 * NH;                 // normalizer warps
-  static constexpr int THREADS = (NWN + 2) * 32;     // + TMA warp + MMA warp
+  // The threshold pass with split rows holds a 64-score chunk, the bucket
+  // maxima and the candidate state per thread: it runs three whole
+  // warpgroups (two idle warps) so that setmaxnreg can move registers from
+  // the TMA / MMA warpgroup to the normalizer warpgroups:
+  // 2 * 128 * 208 + 128 * 88 = 384 * 168, the launch's allocation (the
+  // TMA producer's page walk needs more than 56).
+  static constexpr bool REGSPLIT = (MODE == TC_TAU && NH == 2);
+  static constexpr int REGS_NORM = 208, REGS_CTRL = 88;
+  static constexpr int THREADS = REGSPLIT ? 384 : (NWN + 2) * 32;  // + TMA warp + MMA warp
+  static_assert(!REGSPLIT || 2 * 128 * REGS_NORM + 128 * REGS_CTRL <= 384 * 168,
+                "register split exceeds the launch's allocation");
   static constexpr int QBYTES = D * TC_BM * 2;
   static constexpr int KBYTES = D * BN * 2;
   static constexpr int VBYTES = (MODE == TC_TAU) ? 0 : DV * BN * 2;
@@ -146,12 +163,14 @@ struct TcLayout {
   static constexpr int CAP = TauCap<D>::value;
   static constexpr int CAPR = CAP / NH;         // entries per row half
   static constexpr int CAP_STRIDE = CAPR + 1;    // int2 entries per row half
+  // per row half: CAPR candidates (and one padding entry)
   static constexpr int BUFBYTES = (MODE == TC_TAU) ? CAP_STRIDE * TC_BM * NH * 8 : 0;
-  // split rows in the threshold pass: each half publishes its running lower
-  // bound of the row's threshold for the other half
-  static constexpr int LBXBYTES = (MODE == TC_TAU && NH > 1) ? NH * TC_BM * 4 : 0;
-  static constexpr int OFF_LBX = OFF_BUF + BUFBYTES;
-  static constexpr int OFF_BAR = OFF_LBX + LBXBYTES;
+  // per normalizer thread: the 32 scores of the chunk it is appending from
+  // (and, at the end of the bound pass, its 32 bucket maxima for the other
+  // half of its row)
+  static constexpr int STASHBYTES = (MODE == TC_TAU) ? NWN * 32 * 32 * 4 : 0;
+  static constexpr int OFF_STASH = OFF_BUF + BUFBYTES;
+  static constexpr int OFF_BAR = OFF_STASH + STASHBYTES;
   // S ring depth in TMEM: the threshold pass has no O accumulator, so it
   // keeps four S buffers and its normalizer warps can drift three blocks apart
   static constexpr int NSB = (MODE == TC_TAU) ? 4 : 2;
@@ -237,6 +256,52 @@ __device__ __forceinline__ float thread_row_tau(const int2* row0, int n0, const 
   return t + m;
 }
 
+// Exact threshold of N values held in registers, in shifted threshold units
+// (w = u - m with m the row maximum; -inf for no key), by the Newton
+// iteration of thread_row_tau: every iterate is a lower bound of the
+// threshold.  Returns it in shifted units.
+template <int N>
+__device__ __forceinline__ float reg_row_tau(const float (&w)[N], bool entmax, float t0,
+                                             int max_it = 32) {
+  float t = fmaxf(t0, -1.f);
+  for (int it = 0; it < max_it; ++it) {
+    // two partial sums per statistic shorten the dependent chains
+    float c0 = 0.f, c1 = 0.f, a0 = 0.f, a1 = 0.f, q0 = 0.f, q1 = 0.f;
+    float wmin = INFINITY;
+#pragma unroll
+    for (int i = 0; i < N; i += 2) {
+      const bool in0 = w[i] > t, in1 = w[i + 1] > t;
+      const float x0 = in0 ? w[i] : 0.f, x1 = in1 ? w[i + 1] : 0.f;
+      c0 += in0 ? 1.f : 0.f;
+      c1 += in1 ? 1.f : 0.f;
+      a0 += x0;
+      a1 += x1;
+      q0 = fmaf(x0, x0, q0);
+      q1 = fmaf(x1, x1, q1);
+      wmin = fminf(wmin, fminf(in0 ? w[i] : INFINITY, in1 ? w[i + 1] : INFINITY));
+    }
+    const float cnt = c0 + c1, s1 = a0 + a1, s2 = q0 + q1;
+    float ts, tn;
+    bool valid = true;
+    if (!entmax) {
+      ts = (s1 - 1.f) / cnt;
+      tn = ts;
+    } else {
+      const float mu = s1 / cnt;
+      const float delta = (1.f - (s2 - s1 * mu)) / cnt;
+      valid = delta >= 0.f;
+      ts = valid ? mu - sqrtf(delta) : -INFINITY;
+      const float g = s2 - 2.f * t * s1 + t * t * cnt;
+      const float gp = 2.f * (s1 - t * cnt);
+      tn = t + (g - 1.f) / gp;
+    }
+    if (valid && ts >= t && wmin > ts) return ts;
+    if (!(tn > t)) break;
+    t = tn;
+  }
+  return t;
+}
+
 // Keep the entries above `lb` (threshold units), compacted in place to the
 // front of the row; returns the new count and, in *kept_sum, the sum of the
 // kept stored values.
@@ -257,7 +322,7 @@ __device__ __forceinline__ int thread_compact_row(int2* row, int n, float vscale
 }
 
 template <int D, int DV, int BN, int KST, int VST, int MODE, int NH = 1>
-__global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
+__global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THREADS), 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                       const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, TcArgs A) {
@@ -292,6 +357,8 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
   const int kend = (khi >= klo) ? khi / BN + 1 : kb0;
   // blocks of [kb0, kend) the block mask keeps (all of them without one)
   const int nblk = count_kept<BN>(P, b, h, h, qt, kb0, kend);
+  // S tiles the MMA produces: the threshold pass multiplies every block twice
+  const int nseq = (MODE == TC_TAU) ? 2 * nblk : nblk;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + LY::OFF_BAR);
   const uint32_t bar_q = smem_addr(&bars[0]);
@@ -305,10 +372,6 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + LY::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
 
-  if constexpr (LY::LBXBYTES > 0) {
-    float* lbx = reinterpret_cast<float*>(smem + LY::OFF_LBX);
-    for (int i = tid; i < NH * TC_BM; i += LY::THREADS) lbx[i] = -INFINITY;
-  }
   if (tid == 0) {
     mbar_init(bar_q, 1);
     for (int s = 0; s < KST; ++s) {
@@ -338,6 +401,7 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
 
   if (warp == NWN) {
     // ======================= TMA producer ===================================
+    if constexpr (LY::REGSPLIT) regs_dec<LY::REGS_CTRL>();
     if (lane == 0 && nblk > 0) {
       tma_prefetch_desc(&tmq);
       tma_prefetch_desc(&tmk);
@@ -347,8 +411,11 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
       for (int x = 0; x < D / 64; ++x)
         tma_load_rows(smem_addr(smem + LY::OFF_Q + x * TC_BM * 128), &tmq, bar_q, x * 64,
                       packed ? sq.q0 + q0 : q0, packed ? h : bh, packed);
+      // the threshold pass streams the key blocks twice (bound pass, then
+      // candidate pass)
       int kb = next_kept<BN>(P, b, h, h, qt, kb0, kend);
-      for (int j = 0; j < nblk; ++j, kb = next_kept<BN>(P, b, h, h, qt, kb + 1, kend)) {
+      for (int j = 0; j < nseq; ++j, kb = next_kept<BN>(P, b, h, h, qt, kb + 1, kend)) {
+        if (j == nblk) kb = next_kept<BN>(P, b, h, h, qt, kb0, kend);
         const int ks = j % KST;
         if (j >= KST && !mbar_wait(bar_kempty(ks), ((j / KST) + 1) & 1, abort_flag)) break;
         mbar_expect_tx(bar_kfull(ks), LY::KBYTES);
@@ -366,14 +433,15 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
     }
   } else if (warp == NWN + 1) {
     // ======================= MMA issuer =====================================
+    if constexpr (LY::REGSPLIT) regs_dec<LY::REGS_CTRL>();
     if (lane == 0 && nblk > 0) {
       constexpr uint32_t IDESC_S = idesc_bf16(TC_BM, BN, 0, 0);
       constexpr uint32_t IDESC_O = idesc_bf16(TC_BM, DV, 0, 1);
       const uint32_t qbase = smem_addr(smem + LY::OFF_Q);
       bool ok = mbar_wait_spin(bar_q, 0, abort_flag);
       tc_fence_after();
-      for (int j = 0; ok && j <= nblk; ++j) {
-        if (j < nblk) {
+      for (int j = 0; ok && j <= nseq; ++j) {
+        if (j < nseq) {
           const int sb = j % NSB, ks = j % KST;
           if (!mbar_wait_spin(bar_kfull(ks), (j / KST) & 1, abort_flag)) break;
           // S buffer sb held P_{j-2}.  With a PV product that reads it, that
@@ -427,8 +495,12 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
         }
       }
     }
+  } else if (warp >= NWN + 2) {
+    // idle warps (register split only): they hand their registers over
+    if constexpr (LY::REGSPLIT) regs_dec<LY::REGS_CTRL>();
   } else {
     // ======================= normalizer warps ==============================
+    if constexpr (LY::REGSPLIT) regs_inc<LY::REGS_NORM>();
     const int quarter = warp & 3;        // TMEM lane quarter = query rows
     const int half = warp >> 2;          // which columns of the S row
     const int cbase = half * NC;
@@ -449,15 +521,16 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
     float m_run, l_run = 0.f, tau = 0.f;
     // TAU state
     int2* const bufbase = reinterpret_cast<int2*>(smem + LY::OFF_BUF);
-    volatile float* const lbx_mine = reinterpret_cast<float*>(smem + LY::OFF_LBX) + half * TC_BM + row;
-    volatile float* const lbx_other =
-        reinterpret_cast<float*>(smem + LY::OFF_LBX) + (NH - 1 - half) * TC_BM + row;
-    int2* tbuf = bufbase + (size_t)(half * TC_BM + quarter * 32) * LY::CAP_STRIDE;  // 32 rows
-    int2* mybuf = tbuf + lane * LY::CAP_STRIDE;
+    int2* const mybuf = bufbase + (size_t)(half * TC_BM + row) * LY::CAP_STRIDE;
     int nbuf = 0;
-    float bsum = 0.f;  // sum of the stored values in the buffer
     bool ovf = false;
     float lb = -INFINITY;  // lower bound of tau (threshold units)
+    float thr = -INFINITY; // the same in stored units, less a rounding margin
+    // bound pass: bucket k keeps the largest stored value of the columns
+    // congruent to k mod 32 of this thread's part of the row
+    float bk[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) bk[k] = -INFINITY;
     if constexpr (MODE == TC_ONLINE) {
       // the sink (softmax1's logit 0, or a learned per-head logit, in log2
       // units) belongs to exactly one half of the row
@@ -470,13 +543,66 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
     const bool entmax = P.norm == NATTN_ENTMAX15;
     bool alive = true;
 
-    int kbc = next_kept<BN>(P, b, h, h, qt, kb0, kend);  // key block of step j
-    for (int j = 0; j < nblk; ++j, kbc = next_kept<BN>(P, b, h, h, qt, kbc + 1, kend)) {
-      const int sb = j % NSB;
-      if (!__all_sync(0xffffffffu, mbar_wait_spin(bar_sfull(sb), (j / NSB) & 1, abort_flag))) {
-        alive = false;
-        break;
+    const float vs = fast ? zs : 1.f;  // stored value -> threshold units
+    // candidates are tested in stored units against a bound less a margin far
+    // above the rounding of the bound's arithmetic
+    auto to_thr = [&](float bnd) {
+      const float bm = bnd - (fabsf(bnd) + 1.f) * 4e-6f;
+      return fast ? bm * izs : bm;
+    };
+    // End of the bound pass (threshold mode).  The bucket maxima are distinct
+    // keys of the row, and adding keys to a set only raises its threshold, so
+    // the exact threshold of the bucket set is a lower bound of the row's:
+    // every support key lies above it.  With split rows the two halves swap
+    // their buckets once (through the stash, which the candidate pass uses
+    // only afterwards) and both solve over all of them in registers.
+    auto bound_pass_done = [&]() {
+      constexpr int NB = 32 * NH;  // bucket maxima of the row
+      float w[NB];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) w[k] = bk[k];
+      if constexpr (NH > 1) {
+        // the other half of this thread's row is normalizer thread tid ^ 128
+        static_assert(NWN == 8, "two halves of four warps");
+        constexpr int NT = NWN * 32;
+        float4* const sx = reinterpret_cast<float4*>(smem + LY::OFF_STASH);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          sx[q * NT + tid] = make_float4(bk[4 * q], bk[4 * q + 1], bk[4 * q + 2], bk[4 * q + 3]);
+        asm volatile("bar.sync 1, %0;" ::"r"(NWN * 32) : "memory");
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 x = sx[q * NT + (tid ^ 128)];
+          w[32 + 4 * q] = x.x;
+          w[33 + 4 * q] = x.y;
+          w[34 + 4 * q] = x.z;
+          w[35 + 4 * q] = x.w;
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(NWN * 32) : "memory");
       }
+      float bmax = w[0];
+#pragma unroll
+      for (int k = 1; k + 1 < NB; k += 2) bmax = fmax3(bmax, w[k], w[k + 1]);
+      bmax = fmaxf(bmax, w[NB - 1]);
+      m_run = bmax * vs;  // the row maximum (threshold units)
+      if (m_run == -INFINITY) {
+        lb = thr = -INFINITY;
+        return;
+      }
+#pragma unroll
+      for (int k = 0; k < NB; ++k) w[k] = fmaf(w[k], vs, -m_run);
+      lb = m_run + reg_row_tau<NB>(w, entmax, -1.f);
+      thr = to_thr(lb);
+    };
+
+    static_assert(NC == 64, "each normalizer thread owns 64 columns of a block");
+    // Wait for S(j) and load this thread's 64 scores of key block kbc: z
+    // (threshold / log2 units) unless the fast path keeps raw scores; masked
+    // entries become -inf.  False when the wait was given up.
+    auto load_scores = [&](int j, int kbc, uint32_t(&r)[64]) -> bool {
+      const int sb = j % NSB;
+      if (!__all_sync(0xffffffffu, mbar_wait_spin(bar_sfull(sb), (j / NSB) & 1, abort_flag)))
+        return false;
       tc_fence_after();
       const int jb = kbc * BN + cbase;  // first key of this thread's columns
       const bool edge = !(rr.lo <= jb && rr.hi >= jb + NC - 1);
@@ -487,39 +613,42 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
         klb = NC;
         span = 0;
       }
-      const uint32_t sbase = lane_base + LY::TM_S + sb * BN + cbase;
-      // the online mode needs its whole part of the row at once (maximum
-      // before exponentials); the sparse modes work on 64-key sub-blocks
-      constexpr int LDC = (MODE == TC_ONLINE || NC < 64) ? NC : 64;
-#pragma unroll 1
-      for (int hs = 0; hs < NC / LDC; ++hs) {
-      const uint32_t saddr = sbase + hs * LDC;       // S columns of this sub-block
-      const uint32_t paddr = sbase + hs * (LDC / 2); // packed P columns
-      const int j0 = jb + hs * LDC;
-      const int kl = klb - hs * LDC;
-
-      uint32_t r[LDC];
-#pragma unroll
-      for (int c = 0; c < LDC / 32; ++c)
-        tmem_ld32(saddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+      const uint32_t saddr = lane_base + LY::TM_S + sb * BN + cbase;
+      tmem_ld32(saddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+      tmem_ld32(saddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
       tmem_ld_wait();
-
-      // scores -> z (threshold / log2 units) unless the fast path keeps raw s;
-      // masked entries become -inf
       if (!fast) {
 #pragma unroll
-        for (int k = 0; k < LDC; ++k) r[k] = __float_as_uint(tc_z(__uint_as_float(r[k]), A));
+        for (int k = 0; k < 64; ++k) r[k] = __float_as_uint(tc_z(__uint_as_float(r[k]), A));
       }
       if (edge) {
 #pragma unroll
-        for (int k = 0; k < LDC; ++k)
-          if ((unsigned)(k - kl) > span) r[k] = __float_as_uint(-INFINITY);
+        for (int k = 0; k < 64; ++k)
+          if ((unsigned)(k - klb) > span) r[k] = __float_as_uint(-INFINITY);
       }
+      return true;
+    };
+    // S(j) (or the P written over it) has been read: its buffer is free
+    auto release = [&](int j) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_pfull(j % NSB));
+    };
+    const int kfirst = next_kept<BN>(P, b, h, h, qt, kb0, kend);
 
-      if constexpr (MODE == TC_ONLINE) {
+    if constexpr (MODE == TC_ONLINE) {
+      int kbc = kfirst;  // key block of step j
+      for (int j = 0; j < nblk; ++j, kbc = next_kept<BN>(P, b, h, h, qt, kbc + 1, kend)) {
+        uint32_t r[64];
+        if (!load_scores(j, kbc, r)) {
+          alive = false;
+          break;
+        }
+        const uint32_t paddr = lane_base + LY::TM_S + (j % NSB) * BN + cbase;  // packed P
+
         float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-        for (int k = 0; k < LDC; k += 4) {
+        for (int k = 0; k < 64; k += 4) {
           mx0 = fmaxf(mx0, __uint_as_float(r[k]));
           mx1 = fmaxf(mx1, __uint_as_float(r[k + 1]));
           mx2 = fmaxf(mx2, __uint_as_float(r[k + 2]));
@@ -534,7 +663,6 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
         const float msafe = (m_use == -INFINITY) ? 0.f : m_use;
         const float fa = fast ? zs : 1.f;  // p = exp2(x * fa - msafe)
         float s0 = 0.f, s1 = 0.f;
-        static_assert(LDC == 64, "one 64-score chunk per online step");
         uint32_t pk[32];  // 64 scores -> 32 packed columns
         exp2_pack64(&r[0], fa, msafe, s0, s1, pk);
         // P(j) is stored only once the previous block's PV has completed, so
@@ -565,46 +693,42 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
           tmem_st_wait();
         }
         m_run = m_use;
-      } else {  // TC_TAU
-        const float vs = fast ? zs : 1.f;  // stored value -> threshold units
-        // chunk maxima first: independent of the bound logic below
-        float cmaxs[LDC / 32];
+        release(j);
+      }
+    } else {
+      // bound pass: bucket maxima
+      int kbc = kfirst;
+      for (int j = 0; j < nblk; ++j, kbc = next_kept<BN>(P, b, h, h, qt, kbc + 1, kend)) {
+        uint32_t r[64];
+        if (!load_scores(j, kbc, r)) {
+          alive = false;
+          break;
+        }
 #pragma unroll
-        for (int c = 0; c < LDC / 32; ++c) cmaxs[c] = max32_bits(&r[c * 32]) * vs;
+        for (int k = 0; k < 32; ++k)
+          bk[k] = fmax3(bk[k], __uint_as_float(r[k]), __uint_as_float(r[k + 32]));
+        release(j);
+      }
+      // every normalizer warp takes the bound's named barriers exactly once,
+      // also for a tile without key blocks or after a wait was given up
+      bound_pass_done();
+      // candidate pass: every key above the bound
+      kbc = kfirst;
+      for (int j = nblk; alive && j < nseq; ++j, kbc = next_kept<BN>(P, b, h, h, qt, kbc + 1, kend)) {
+        uint32_t r[64];
+        if (!load_scores(j, kbc, r)) {
+          alive = false;
+          break;
+        }
+        const int j0 = kbc * BN + cbase;  // key of column 0
+
 #pragma unroll
-        for (int c = 0; c < LDC / 32; ++c) {
+        for (int c = 0; c < 2; ++c) {
           const uint32_t* rc = &r[c * 32];
-          const float cmax = cmaxs[c];
-          m_run = fmaxf(m_run, cmax);
-          lb = fmaxf(lb, m_run - 1.f);  // tau >= max - 1
-          // The buffer B holds every stored key that can still be in the
-          // support, so for the threshold of the keys seen so far
-          //   sparsemax: sum_B (u - tau) <= 1          -> tau >= (sum u - 1)/|B|
-          //   entmax15:  sum_B (u - tau) <= sqrt(|B|)  -> tau >= mean u - 1/sqrt|B|
-          // (Cauchy-Schwarz with sum_S (u - tau)^2 = 1); adding keys only
-          // raises tau, so either is a valid running lower bound.
-          if (nbuf > 0) {
-            const float fn = (float)nbuf;
-            const float su = bsum * vs;
-            lb = fmaxf(lb, entmax ? __fdividef(su, fn) - rsqrtf(fn) : __fdividef(su - 1.f, fn));
-          }
-          if constexpr (NH > 1) {
-            // a bound of one half's keys bounds the whole row; a stale read
-            // of the other half's value is still a valid bound
-            lb = fmaxf(lb, lbx_other[0]);
-            lbx_mine[0] = lb;
-          }
-          const bool want = cmax > lb && !ovf;
+          const bool want = max32_bits(rc) > thr && !ovf;
           if (!__any_sync(0xffffffffu, want)) continue;
-          // candidates are tested in stored units against the bound less a
-          // margin far above the rounding of the bound's arithmetic
-          auto to_thr = [&](float b) {
-            const float bm = b - (fabsf(b) + 1.f) * 4e-6f;
-            return fast ? bm * izs : bm;
-          };
-          float thr = to_thr(lb);
-          // candidate mask: bit k set when value k is above thr, taken from
-          // the sign of thr - v (-inf values give +inf: never candidates)
+          // candidate mask: bit k set when value k is above t, taken from the
+          // sign of t - v (-inf values give +inf: never candidates)
           // (four independent eight-bit chains, merged at the end)
           auto cand_mask = [&](float t) {
             unsigned part[4];
@@ -619,18 +743,24 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
             return part[0] | (part[1] << 8) | (part[2] << 16) | (part[3] << 24);
           };
           unsigned msk = want ? cand_mask(thr) : 0u;
-          // the chunk goes to a per-thread stash so that appends run once per
-          // candidate, not once per key
-          float stash[32];
+          // the chunk goes to this thread's stash in shared memory so that
+          // appends run once per candidate, not once per key (16-byte
+          // pieces interleaved across the normalizer threads: conflict-free
+          // stores; a thread reads back only what it wrote)
+          constexpr int NT = NWN * 32;
+          float* const sst = reinterpret_cast<float*>(smem + LY::OFF_STASH);
 #pragma unroll
-          for (int k = 0; k < 32; ++k) stash[k] = __uint_as_float(rc[k]);
+          for (int q = 0; q < 8; ++q)
+            reinterpret_cast<float4*>(sst)[q * NT + tid] =
+                make_float4(__uint_as_float(rc[4 * q]), __uint_as_float(rc[4 * q + 1]),
+                            __uint_as_float(rc[4 * q + 2]), __uint_as_float(rc[4 * q + 3]));
+          auto stash = [&](int k) { return sst[((k >> 2) * NT + tid) * 4 + (k & 3)]; };
           const int kj = j0 + c * 32;
-          // append candidates (lowest key first) while there is room; stored
-          // values are compared in stored units, and a key a rounding step
-          // below the bound is harmless (the exact solve drops it)
+          // append candidates (lowest key first) while there is room; a key a
+          // rounding step below the bound is harmless (the exact solve drops
+          // it)
           auto append = [&](int room) {
             int2* ptr = mybuf + nbuf;
-            float sadd = 0.f;
             int na = 0;
             // two candidates per trip, so that two stash loads are in flight
             while (msk && na + 1 < room) {
@@ -638,61 +768,52 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
               msk &= msk - 1;
               const int k1 = msk ? __ffs(msk) - 1 : -1;
               msk &= msk - 1;  // no-op when msk is already 0
-              const float v0 = stash[k0];
-              const float v1 = (k1 >= 0) ? stash[k1] : 0.f;
+              const float v0 = stash(k0);
+              const float v1 = (k1 >= 0) ? stash(k1) : 0.f;
               *ptr = make_int2(kj + k0, __float_as_int(v0));
               if (k1 >= 0) ptr[1] = make_int2(kj + k1, __float_as_int(v1));
               ptr += (k1 >= 0) ? 2 : 1;
-              sadd += v0 + v1;
               na += (k1 >= 0) ? 2 : 1;
             }
             if (msk && na < room) {  // room for one more
               const int k = __ffs(msk) - 1;
               msk &= msk - 1;
-              const float v = stash[k];
-              *ptr++ = make_int2(kj + k, __float_as_int(v));
-              sadd += v;
+              *ptr++ = make_int2(kj + k, __float_as_int(stash(k)));
               ++na;
             }
             nbuf += na;
-            bsum += sadd;
           };
-          // when a row's buffer cannot take this chunk's candidates, every row
-          // of the warp raises its bound by one Newton step towards the
-          // threshold of the keys it has seen and compacts (each thread its
-          // own row, side by side: the rows of a tile fill their buffers at
-          // similar rates, so one batch stands in for many single-row solves;
-          // one step measured faster than two or than solving exactly)
+          // when a row's buffer cannot take this chunk's candidates (a support
+          // far wider than the bucket set), every row of the warp raises its
+          // bound by one Newton step towards the threshold of the keys it has
+          // kept and compacts (each thread its own row, side by side); if the
+          // candidates still do not fit, the exact threshold is taken with them
+          // included, a few rounds at most, and only then is the row listed
+          // for the row-wise pass
           if (__any_sync(0xffffffffu, nbuf + __popc(msk) > LY::CAPR)) {
+            float ksum;
             lb = fmaxf(lb, thread_row_tau(mybuf, nbuf, mybuf, 0, vs, m_run, entmax, lb - m_run, 1));
-            nbuf = thread_compact_row(mybuf, nbuf, vs, lb, &bsum);
+            nbuf = thread_compact_row(mybuf, nbuf, vs, lb, &ksum);
             thr = to_thr(lb);
             msk &= cand_mask(thr);
-            // still too many: take candidates until the buffer is full and
-            // solve again with them included (they are seen keys too), a few
-            // rounds at most; a row that still cannot fit goes to the
-            // row-wise pass
             for (int round = 0; round < 4 && nbuf + __popc(msk) > LY::CAPR; ++round) {
               append(LY::CAPR - nbuf);
               lb = fmaxf(lb, thread_row_tau(mybuf, nbuf, mybuf, 0, vs, m_run, entmax, lb - m_run));
-              nbuf = thread_compact_row(mybuf, nbuf, vs, lb, &bsum);
-              msk &= cand_mask(to_thr(lb));
+              nbuf = thread_compact_row(mybuf, nbuf, vs, lb, &ksum);
+              thr = to_thr(lb);
+              msk &= cand_mask(thr);
             }
             if (nbuf + __popc(msk) > LY::CAPR) {
               ovf = true;
               msk = 0;
             }
-            if constexpr (NH > 1) lbx_mine[0] = lb;
           }
           if (__any_sync(0xffffffffu, msk != 0)) append(32);
         }
+        release(j);
       }
-      }  // sub-blocks
-      if (!alive) break;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_pfull(sb));
     }
+
 
     // ---- epilogue ----------------------------------------------------------
     if constexpr (MODE == TC_TAU) {
@@ -700,7 +821,6 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
       // with split rows the two halves' buffers are merged (each half's
       // bound is a valid bound of the whole row's threshold) and the row's
       // two warps take one half of the quarter's rows each
-      const float vs = fast ? zs : 1.f;
       float m_r = m_run, lb_r = lb;
       int n0 = nbuf, n1 = 0;
       bool ovf_r = ovf, mine = true;
@@ -865,27 +985,53 @@ __global__ void __launch_bounds__(GATHER_WARPS * 32)
     // support entries carry the value row of each key (see value_row)
     const bf16* vbase = P.v + lane * PER;
     const int2* lst = sup_list + flat * (size_t)sup_cap;
+    // four support rows per step, their loads issued before any is used
+    auto fma_row = [&](float p, const bf16* vr) {
+      if constexpr (PER == 8) {
+        const uint4 x = *reinterpret_cast<const uint4*>(vr);
+        acc[0] += p * bf16lo(x.x); acc[1] += p * bf16hi(x.x);
+        acc[2] += p * bf16lo(x.y); acc[3] += p * bf16hi(x.y);
+        acc[4] += p * bf16lo(x.z); acc[5] += p * bf16hi(x.z);
+        acc[6] += p * bf16lo(x.w); acc[7] += p * bf16hi(x.w);
+      } else if constexpr (PER == 4) {
+        const uint2 x = *reinterpret_cast<const uint2*>(vr);
+        acc[0] += p * bf16lo(x.x); acc[1] += p * bf16hi(x.x);
+        acc[2] += p * bf16lo(x.y); acc[3] += p * bf16hi(x.y);
+      } else {
+        const uint32_t x = *reinterpret_cast<const uint32_t*>(vr);
+        acc[0] += p * bf16lo(x); acc[1] += p * bf16hi(x);
+      }
+    };
     for (int e0 = 0; e0 < n; e0 += 32) {
       const int2 mine = (e0 + lane < n) ? lst[e0 + lane] : make_int2(0, 0);
       const int cnt = min(32, n - e0);
-      for (int e = 0; e < cnt; ++e) {
+      int e = 0;
+      for (; e + 4 <= cnt; e += 4) {
+        int j[4];
+        float p[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          j[u] = __shfl_sync(0xffffffffu, mine.x, e + u);
+          p[u] = __int_as_float(__shfl_sync(0xffffffffu, mine.y, e + u));
+        }
+        if constexpr (PER == 4) {
+          uint2 x[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) x[u] = *reinterpret_cast<const uint2*>(vbase + (size_t)j[u] * DV);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            acc[0] += p[u] * bf16lo(x[u].x); acc[1] += p[u] * bf16hi(x[u].x);
+            acc[2] += p[u] * bf16lo(x[u].y); acc[3] += p[u] * bf16hi(x[u].y);
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) fma_row(p[u], vbase + (size_t)j[u] * DV);
+        }
+      }
+      for (; e < cnt; ++e) {
         const int j = __shfl_sync(0xffffffffu, mine.x, e);
         const float p = __int_as_float(__shfl_sync(0xffffffffu, mine.y, e));
-        const bf16* vr = vbase + (size_t)j * DV;
-        if constexpr (PER == 8) {
-          const uint4 x = *reinterpret_cast<const uint4*>(vr);
-          acc[0] += p * bf16lo(x.x); acc[1] += p * bf16hi(x.x);
-          acc[2] += p * bf16lo(x.y); acc[3] += p * bf16hi(x.y);
-          acc[4] += p * bf16lo(x.z); acc[5] += p * bf16hi(x.z);
-          acc[6] += p * bf16lo(x.w); acc[7] += p * bf16hi(x.w);
-        } else if constexpr (PER == 4) {
-          const uint2 x = *reinterpret_cast<const uint2*>(vr);
-          acc[0] += p * bf16lo(x.x); acc[1] += p * bf16hi(x.x);
-          acc[2] += p * bf16lo(x.y); acc[3] += p * bf16hi(x.y);
-        } else {
-          const uint32_t x = *reinterpret_cast<const uint32_t*>(vr);
-          acc[0] += p * bf16lo(x); acc[1] += p * bf16hi(x);
-        }
+        fma_row(p, vbase + (size_t)j * DV);
       }
     }
   }
