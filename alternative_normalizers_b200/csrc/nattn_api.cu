@@ -155,7 +155,7 @@ struct Plan {
   int R = 0, nsplit = 0, pps = 0;
   // scratch offsets (bytes)
   size_t off_tau = 0, off_ovfc = 0, off_ovfr = 0, off_slots = 0;
-  size_t off_supc = 0, off_supl = 0;
+  size_t off_supc = 0, off_supl = 0, off_rlb = 0;
   int sup_cap = 0;
   size_t off_opart = 0, off_ml = 0, off_scores = 0, off_pmask = 0;
   int pm_words = 0;
@@ -270,7 +270,9 @@ Plan make_plan(const nattn_args* a) {
       pl.off_ovfr = off;
       off = up256(off + rows * 4);
       pl.sup_cap = (a->d >= 256) ? TauCap<256>::value : TauCap<128>::value;
-      pl.off_supc = off;
+      pl.off_supc = off;  // one count per row half
+      off = up256(off + rows * 2 * 4);
+      pl.off_rlb = off;
       off = up256(off + rows * 4);
       pl.off_supl = off;
       off = up256(off + rows * (size_t)pl.sup_cap * 8);
@@ -390,6 +392,7 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
     A.sup_count = nullptr;
     A.sup_list = nullptr;
     A.sup_cap = 0;
+    A.rlb = nullptr;
     // two query heads of one KV group per CTA, each with its own S and O
     if constexpr (D <= 128) {
       if ((a->Hq / a->Hkv) % 2 == 0) {
@@ -433,30 +436,33 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
   A.ovf_rows = reinterpret_cast<int*>(ws + pl.off_ovfr);
   A.sup_count = reinterpret_cast<int*>(ws + pl.off_supc);
   A.sup_list = reinterpret_cast<int2*>(ws + pl.off_supl);
+  A.rlb = reinterpret_cast<float*>(ws + pl.off_rlb);
   A.sup_cap = pl.sup_cap;
   if (cudaMemsetAsync(A.ovf_count, 0, sizeof(int), st) != cudaSuccess) return NATTN_ECUDA;
-  // support sizes start at zero: the gather reads every row, and rows that
-  // no sequence owns (packed padding, a sequence rejected on the device) are
-  // never written by the threshold pass
-  if (cudaMemsetAsync(A.sup_count, 0, (size_t)num_rows(a) * sizeof(int), st) != cudaSuccess)
+  // d <= 128: each S row split between two warps (eight normalizer warps
+  // hide each other's latency); d = 256 keeps whole rows (64-key blocks
+  // leave 32 columns per half)
+  constexpr int NHT = (D <= 128) ? 2 : 1;
+  using LY = TcLayout<D, D, BN, 2, 1, TC_TAU, NHT>;
+  static_assert(LY::CAP == TauCap<(D >= 256 ? 256 : 128)>::value, "workspace plan capacity");
+  // candidate counts start at zero: the apply kernel reads every row, and
+  // rows that no sequence owns (packed padding, a sequence rejected on the
+  // device) are never written by the threshold pass
+  if (cudaMemsetAsync(A.sup_count, 0, (size_t)num_rows(a) * NHT * sizeof(int), st) !=
+      cudaSuccess)
     return NATTN_ECUDA;
   {
-    // d <= 128: each S row split between two warps (eight normalizer warps
-    // hide each other's latency; the halves share their bounds); d = 256
-    // keeps whole rows (64-key blocks leave 32 columns per half)
-    constexpr int NHT = (D <= 128) ? 2 : 1;
-    using LY = TcLayout<D, D, BN, 2, 1, TC_TAU, NHT>;
     auto k = prefill_tc_kernel<D, D, BN, 2, 1, TC_TAU, NHT>;
     if (allow_smem(k, LY::ALLOC) != cudaSuccess) return NATTN_ECUDA;
     k<<<grid, LY::THREADS, LY::ALLOC, st>>>(mq, mk, mv, A);
     if (check_launch() != NATTN_OK) return NATTN_ECUDA;
   }
   {
-    // phase 2: fp32 gather over each row's support list
+    // phase 2: exact threshold and fp32 gather, one warp per row
     const size_t rows = (size_t)num_rows(a);
-    const unsigned g2 = (unsigned)((rows + GATHER_WARPS - 1) / GATHER_WARPS);
-    sparse_gather_kernel<D><<<g2, GATHER_WARPS * 32, 0, st>>>(P, A.sup_count, A.sup_list,
-                                                              A.sup_cap, A.tau);
+    const unsigned g2 = (unsigned)((rows + APPLY_WARPS - 1) / APPLY_WARPS);
+    sparse_apply_kernel<D, NHT, LY::CAPR><<<g2, APPLY_WARPS * 32, 0, st>>>(
+        P, A.sup_count, A.sup_list, A.tau, A.rlb);
     if (check_launch() != NATTN_OK) return NATTN_ECUDA;
   }
   // rows whose candidate buffer overflowed: exact row-wise recomputation

@@ -39,8 +39,8 @@
 //           the CUDA cores, which sets this mode's speed.  Rows whose
 //           candidates overflow the buffer are listed for the row-wise
 //           kernel.
-// Sparse phase 2 is sparse_gather_kernel below: an fp32 sum over each row's
-// support list.
+// Sparse phase 2 is sparse_apply_kernel below: each row's exact threshold
+// from its candidates, then an fp32 sum over its support.
 #pragma once
 
 #include "common.cuh"
@@ -64,11 +64,13 @@ struct TcArgs {
   Problem P;
   float zscale;      // ONLINE: scale * log2(e); TAU: scale * uscale
   float capscale;    // soft-cap: z = capscale * tanh(s * scale / cap)
-  float* tau;        // [B*Hq*Tq]: written by TAU, read by the gather
+  float* tau;        // [rows] TAU: the row maximum (threshold units)
   int* ovf_rows;     // TAU: rows whose candidate buffer overflowed
   int* ovf_count;    // TAU: number of such rows (zeroed before the launch)
-  int* sup_count;    // TAU: support size of every row (0 for overflowed rows)
-  int2* sup_list;    // TAU: [rows][sup_cap] (value row of the key, weight bits)
+  int* sup_count;    // TAU: [rows][halves] candidate counts (-1: the row overflowed)
+  int2* sup_list;    // TAU: [rows][halves][sup_cap / halves] (value row of the key,
+                     //      value less the row maximum in threshold units)
+  float* rlb;        // TAU: [rows] lower bound of the threshold less the row maximum
   int sup_cap;
 };
 
@@ -300,6 +302,12 @@ __device__ __forceinline__ float reg_row_tau(const float (&w)[N], bool entmax, f
     t = tn;
   }
   return t;
+}
+
+// Weight of a support key from its excess x = u - tau > 0 over the
+// threshold: x for sparsemax, x^2 for 1.5-entmax.
+__device__ __forceinline__ float entmax_weight(float x, const Problem& P) {
+  return P.norm == NATTN_ENTMAX15 ? x * x : x;
 }
 
 // Keep the entries above `lb` (threshold units), compacted in place to the
@@ -817,55 +825,42 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
 
     // ---- epilogue ----------------------------------------------------------
     if constexpr (MODE == TC_TAU) {
-      // exact tau and the support list of every row, one thread per row;
-      // with split rows the two halves' buffers are merged (each half's
-      // bound is a valid bound of the whole row's threshold) and the row's
-      // two warps take one half of the quarter's rows each
-      float m_r = m_run, lb_r = lb;
-      int n0 = nbuf, n1 = 0;
-      bool ovf_r = ovf, mine = true;
-      const int2* b0 = mybuf;
-      const int2* b1 = mybuf;
+      // Each row half writes its candidates out as they are (value row of
+      // the key, value less the row maximum in threshold units); the apply
+      // kernel solves every row's exact threshold with a warp per row and
+      // gathers its support.  A row whose candidates overflowed in either
+      // half is listed for the row-wise pass instead.
+      bool ovf_r = ovf;
+      float lb_r = lb;
       if constexpr (NH > 1) {
-        float4* xs = reinterpret_cast<float4*>(smem + LY::OFF_Q);  // Q is no longer read
-        xs[half * TC_BM + row] = make_float4(m_run, lb, __int_as_float(nbuf), ovf ? 1.f : 0.f);
+        float2* xs = reinterpret_cast<float2*>(smem + LY::OFF_Q);  // Q is no longer read
+        xs[half * TC_BM + row] = make_float2(lb, ovf ? 1.f : 0.f);
         asm volatile("bar.sync 1, %0;" ::"r"(NWN * 32) : "memory");
-        const float4 a0 = xs[row], a1 = xs[TC_BM + row];
-        m_r = fmaxf(a0.x, a1.x);
-        lb_r = fmaxf(a0.y, a1.y);
-        n0 = __float_as_int(a0.z);
-        n1 = __float_as_int(a1.z);
-        ovf_r = a0.w != 0.f || a1.w != 0.f;
-        b0 = bufbase + (size_t)row * LY::CAP_STRIDE;
-        b1 = bufbase + (size_t)(TC_BM + row) * LY::CAP_STRIDE;
-        mine = (lane >> 4) == half;
+        const float2 o = xs[(NH - 1 - half) * TC_BM + row];
+        lb_r = fmaxf(lb, o.x);  // both halves' bounds bound the row
+        ovf_r = ovf || o.y != 0.f;
       }
-      if (row_ok && mine) {
-        float t = INFINITY;
-        int nsup = 0;
+      if (row_ok) {
+        const size_t seg = flat * NH + half;
         if (ovf_r) {
-          const int slot = atomicAdd(A.ovf_count, 1);
-          A.ovf_rows[slot] = (int)flat;
-        } else if (m_r != -INFINITY) {
-          t = thread_row_tau(b0, n0, b1, n1, vs, m_r, entmax, lb_r - m_r);
-          int2* dst = A.sup_list + flat * (size_t)A.sup_cap;
-          auto emit = [&](const int2* src, int n) {
-            for (int i = 0; i < n; ++i) {
-              const int2 e = src[i];
-              const float x = __int_as_float(e.y) * vs - t;
-              // the gather reads the support key's value row by its row index
-              if (x > 0.f)
-                dst[nsup++] =
-                    make_int2(value_row(P, b, g, e.x, sq), __float_as_int(entmax ? x * x : x));
-            }
-          };
-          emit(b0, n0);
-          emit(b1, n1);
+          if (half == 0) {
+            const int slot = atomicAdd(A.ovf_count, 1);
+            A.ovf_rows[slot] = (int)flat;
+          }
+          A.sup_count[seg] = -1;
+        } else {
+          int2* dst = A.sup_list + seg * LY::CAPR;
+          for (int i = 0; i < nbuf; ++i) {
+            const int2 e = mybuf[i];
+            dst[i] = make_int2(value_row(P, b, g, e.x, sq),
+                               __float_as_int(fmaf(__int_as_float(e.y), vs, -m_run)));
+          }
+          A.sup_count[seg] = nbuf;
         }
-        A.tau[flat] = t;
-        A.sup_count[flat] = nsup;
-        // rows sent to the row-wise pass get their count there
-        if (!ovf_r && P.row_nnz) P.row_nnz[flat] = nsup;
+        if (half == 0) {
+          A.tau[flat] = m_run;         // row maximum (threshold units)
+          A.rlb[flat] = lb_r - m_run;  // a lower bound of tau less it
+        }
       }
     } else {
       const bool have_o =
@@ -955,91 +950,173 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
 }
 
 
-// Sparse phase 2 (default): O = sum over the row's support of p_j V_j, in
-// fp32 on CUDA cores, from the (value row, weight) list the threshold pass
-// wrote.
-// The support of sparsemax / 1.5-entmax is a handful of keys per row, so
-// this touches |support| value rows instead of multiplying every block, and
-// the weights enter the sum in full precision.  One warp per query row; lane
-// l owns columns [l * dv/32, (l+1) * dv/32).
-constexpr int GATHER_WARPS = 4;
+// Sparse phase 2: one warp per query row.  The row's candidates (every key
+// above a lower bound of its threshold, written by the threshold pass) give
+// the exact threshold by the Newton iteration of thread_row_tau, with the
+// sums taken across the warp; then O = sum over the support of p_j V_j in
+// fp32 on CUDA cores.  The support of sparsemax / 1.5-entmax is a handful of
+// keys per row, so this reads |support| value rows instead of multiplying
+// every block, and the weights enter the sum in full precision.  Lane l
+// owns output columns [l * dv/32, (l+1) * dv/32).
+constexpr int APPLY_WARPS = 4;
 
-template <int DV>
-__global__ void __launch_bounds__(GATHER_WARPS * 32)
-    sparse_gather_kernel(Problem P, const int* __restrict__ sup_count,
-                         const int2* __restrict__ sup_list, int sup_cap,
-                         const float* __restrict__ tau) {
-  constexpr int PER = DV / 32;  // columns per lane (2, 4 or 8)
-  const int lane = threadIdx.x & 31;
+template <int DV, int NSEG, int CAPR>
+__global__ void __launch_bounds__(APPLY_WARPS * 32)
+    sparse_apply_kernel(Problem P, const int* __restrict__ sup_count,
+                        const int2* __restrict__ sup_list, const float* __restrict__ rmax,
+                        const float* __restrict__ rlb) {
+  constexpr int PER = DV / 32;                  // columns per lane (2, 4 or 8)
+  constexpr int NCAND = NSEG * CAPR;            // candidates a row can have
+  constexpr int NE = (NCAND + 31) / 32;         // candidate slots per lane
+  __shared__ int2 sup[APPLY_WARPS][NCAND];      // (value row, weight) of the support
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const size_t rows =
       P.cu_q != nullptr ? (size_t)P.total_q * P.Hq : (size_t)P.B * P.Hq * P.Tq;
-  const size_t flat = (size_t)blockIdx.x * GATHER_WARPS + (threadIdx.x >> 5);
+  const size_t flat = (size_t)blockIdx.x * APPLY_WARPS + wid;
   if (flat >= rows) return;
   // packed: rows past the last sequence belong to no sequence
   if (P.cu_q != nullptr && flat >= (size_t)min(P.cu_q[P.B], P.total_q) * P.Hq) return;
-  const int n = min(sup_count[flat], sup_cap);
+  int c[NSEG];
+  bool ovf = false;
+#pragma unroll
+  for (int sg = 0; sg < NSEG; ++sg) {
+    c[sg] = sup_count[flat * NSEG + sg];
+    ovf |= c[sg] < 0;
+    c[sg] = min(c[sg], CAPR);
+  }
+  if (ovf) return;  // the row-wise pass writes this row
+  // slot r of lane l holds entry r * 32 + l of the concatenated segments
+  const int2* lst = sup_list + flat * NCAND;
+  float w[NE];
+  int vr[NE];
+  int ntot = 0;
+#pragma unroll
+  for (int sg = 0; sg < NSEG; ++sg) ntot += c[sg];
+#pragma unroll
+  for (int r = 0; r < NE; ++r) {
+    const int e = r * 32 + lane;
+    int at = -1;
+    if (e < c[0]) {
+      at = e;
+    } else if constexpr (NSEG > 1) {
+      if (e - c[0] < c[1]) at = CAPR + (e - c[0]);
+    }
+    const int2 x = (at >= 0) ? lst[at] : make_int2(0, __float_as_int(-INFINITY));
+    vr[r] = x.x;
+    w[r] = __int_as_float(x.y);
+  }
+  float tau = INFINITY;  // less the row maximum
+  if (ntot > 0) {
+    const bool entmax = P.norm == NATTN_ENTMAX15;
+    float t = fmaxf(rlb[flat], -1.f);
+    for (int it = 0; it < 64; ++it) {
+      float cnt = 0.f, s1 = 0.f, s2 = 0.f, wmin = INFINITY;
+#pragma unroll
+      for (int r = 0; r < NE; ++r) {
+        if (w[r] > t) {
+          cnt += 1.f;
+          s1 += w[r];
+          s2 = fmaf(w[r], w[r], s2);
+          wmin = fminf(wmin, w[r]);
+        }
+      }
+      // xor butterflies: every lane ends with the same sums
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, off);
+        s2 += __shfl_xor_sync(0xffffffffu, s2, off);
+        wmin = fminf(wmin, __shfl_xor_sync(0xffffffffu, wmin, off));
+      }
+      float ts, tn;
+      bool valid = true;
+      if (!entmax) {
+        ts = (s1 - 1.f) / cnt;
+        tn = ts;
+      } else {
+        const float mu = s1 / cnt;
+        const float delta = (1.f - (s2 - s1 * mu)) / cnt;
+        valid = delta >= 0.f;
+        ts = valid ? mu - sqrtf(delta) : -INFINITY;
+        const float gv = s2 - 2.f * t * s1 + t * t * cnt;
+        const float gp = 2.f * (s1 - t * cnt);
+        tn = t + (gv - 1.f) / gp;
+      }
+      if (valid && ts >= t && wmin > ts) {
+        t = ts;
+        break;
+      }
+      if (!(tn > t)) break;
+      t = tn;
+    }
+    tau = t;
+  }
+  // the support, compacted in candidate order into this warp's list
+  int nsup = 0;
+  const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int r = 0; r < NE; ++r) {
+    const float x = w[r] - tau;
+    const bool in = x > 0.f;
+    const unsigned bal = __ballot_sync(0xffffffffu, in);
+    if (in)
+      sup[wid][nsup + __popc(bal & lt)] = make_int2(vr[r], __float_as_int(entmax_weight(x, P)));
+    nsup += __popc(bal);
+  }
+  __syncwarp();
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  if (n > 0) {
-    // support entries carry the value row of each key (see value_row)
-    const bf16* vbase = P.v + lane * PER;
-    const int2* lst = sup_list + flat * (size_t)sup_cap;
-    // four support rows per step, their loads issued before any is used
-    auto fma_row = [&](float p, const bf16* vr) {
-      if constexpr (PER == 8) {
-        const uint4 x = *reinterpret_cast<const uint4*>(vr);
-        acc[0] += p * bf16lo(x.x); acc[1] += p * bf16hi(x.x);
-        acc[2] += p * bf16lo(x.y); acc[3] += p * bf16hi(x.y);
-        acc[4] += p * bf16lo(x.z); acc[5] += p * bf16hi(x.z);
-        acc[6] += p * bf16lo(x.w); acc[7] += p * bf16hi(x.w);
-      } else if constexpr (PER == 4) {
-        const uint2 x = *reinterpret_cast<const uint2*>(vr);
-        acc[0] += p * bf16lo(x.x); acc[1] += p * bf16hi(x.x);
-        acc[2] += p * bf16lo(x.y); acc[3] += p * bf16hi(x.y);
-      } else {
-        const uint32_t x = *reinterpret_cast<const uint32_t*>(vr);
-        acc[0] += p * bf16lo(x); acc[1] += p * bf16hi(x);
-      }
-    };
-    for (int e0 = 0; e0 < n; e0 += 32) {
-      const int2 mine = (e0 + lane < n) ? lst[e0 + lane] : make_int2(0, 0);
-      const int cnt = min(32, n - e0);
-      int e = 0;
-      for (; e + 4 <= cnt; e += 4) {
-        int j[4];
-        float p[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          j[u] = __shfl_sync(0xffffffffu, mine.x, e + u);
-          p[u] = __int_as_float(__shfl_sync(0xffffffffu, mine.y, e + u));
-        }
-        if constexpr (PER == 4) {
-          uint2 x[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) x[u] = *reinterpret_cast<const uint2*>(vbase + (size_t)j[u] * DV);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            acc[0] += p[u] * bf16lo(x[u].x); acc[1] += p[u] * bf16hi(x[u].x);
-            acc[2] += p[u] * bf16lo(x[u].y); acc[3] += p[u] * bf16hi(x[u].y);
-          }
-        } else {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) fma_row(p[u], vbase + (size_t)j[u] * DV);
-        }
-      }
-      for (; e < cnt; ++e) {
-        const int j = __shfl_sync(0xffffffffu, mine.x, e);
-        const float p = __int_as_float(__shfl_sync(0xffffffffu, mine.y, e));
-        fma_row(p, vbase + (size_t)j * DV);
-      }
+  const bf16* vbase = P.v + lane * PER;
+  auto fma_row = [&](float p, const bf16* vr_) {
+    if constexpr (PER == 8) {
+      const uint4 x = *reinterpret_cast<const uint4*>(vr_);
+      acc[0] += p * bf16lo(x.x); acc[1] += p * bf16hi(x.x);
+      acc[2] += p * bf16lo(x.y); acc[3] += p * bf16hi(x.y);
+      acc[4] += p * bf16lo(x.z); acc[5] += p * bf16hi(x.z);
+      acc[6] += p * bf16lo(x.w); acc[7] += p * bf16hi(x.w);
+    } else if constexpr (PER == 4) {
+      const uint2 x = *reinterpret_cast<const uint2*>(vr_);
+      acc[0] += p * bf16lo(x.x); acc[1] += p * bf16hi(x.x);
+      acc[2] += p * bf16lo(x.y); acc[3] += p * bf16hi(x.y);
+    } else {
+      const uint32_t x = *reinterpret_cast<const uint32_t*>(vr_);
+      acc[0] += p * bf16lo(x); acc[1] += p * bf16hi(x);
     }
+  };
+  // eight value rows per step, their loads issued before any is used
+  int e = 0;
+  for (; e + 8 <= nsup; e += 8) {
+    int2 en[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) en[u] = sup[wid][e + u];
+    if constexpr (PER == 4) {
+      uint2 x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = *reinterpret_cast<const uint2*>(vbase + (size_t)en[u].x * DV);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float p = __int_as_float(en[u].y);
+        acc[0] += p * bf16lo(x[u].x); acc[1] += p * bf16hi(x[u].x);
+        acc[2] += p * bf16lo(x[u].y); acc[3] += p * bf16hi(x[u].y);
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) fma_row(__int_as_float(en[u].y), vbase + (size_t)en[u].x * DV);
+    }
+  }
+  for (; e < nsup; ++e) {
+    const int2 en = sup[wid][e];
+    fma_row(__int_as_float(en.y), vbase + (size_t)en.x * DV);
   }
   bf16* o = P.out + flat * DV + lane * PER;
 #pragma unroll
-  for (int e = 0; e < PER; e += 2)
-    *reinterpret_cast<uint32_t*>(o + e) = pack_bf16(acc[e], acc[e + 1]);
-  if (lane == 0 && P.row_stat) P.row_stat[flat] = tau[flat];
+  for (int k = 0; k < PER; k += 2)
+    *reinterpret_cast<uint32_t*>(o + k) = pack_bf16(acc[k], acc[k + 1]);
+  if (lane == 0) {
+    if (P.row_stat) P.row_stat[flat] = (ntot > 0) ? rmax[flat] + tau : INFINITY;
+    if (P.row_nnz) P.row_nnz[flat] = nsup;
+  }
 }
 
 }  // namespace nattn
