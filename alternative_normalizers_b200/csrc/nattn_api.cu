@@ -458,11 +458,19 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
     if (check_launch() != NATTN_OK) return NATTN_ECUDA;
   }
   {
-    // phase 2: exact threshold and fp32 gather, one warp per row
+    // phase 2: exact threshold and fp32 gather; sparsemax's short supports
+    // are bound by the dependent steps (two rows per warp), 1.5-entmax's by
+    // the value-row loads in flight (one row per warp)
     const size_t rows = (size_t)num_rows(a);
-    const unsigned g2 = (unsigned)((rows + APPLY_WARPS - 1) / APPLY_WARPS);
-    sparse_apply_kernel<D, NHT, LY::CAPR><<<g2, APPLY_WARPS * 32, 0, st>>>(
-        P, A.sup_count, A.sup_list, A.tau, A.rlb);
+    if (a->normalizer == NATTN_SPARSEMAX) {
+      const unsigned g2 = (unsigned)((rows + 2 * APPLY_WARPS - 1) / (2 * APPLY_WARPS));
+      sparse_apply_kernel<D, NHT, LY::CAPR, 2><<<g2, APPLY_WARPS * 32, 0, st>>>(
+          P, A.sup_count, A.sup_list, A.tau, A.rlb);
+    } else {
+      const unsigned g2 = (unsigned)((rows + APPLY_WARPS - 1) / APPLY_WARPS);
+      sparse_apply_kernel<D, NHT, LY::CAPR, 1><<<g2, APPLY_WARPS * 32, 0, st>>>(
+          P, A.sup_count, A.sup_list, A.tau, A.rlb);
+    }
     if (check_launch() != NATTN_OK) return NATTN_ECUDA;
   }
   // rows whose candidate buffer overflowed: exact row-wise recomputation

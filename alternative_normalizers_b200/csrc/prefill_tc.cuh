@@ -174,19 +174,25 @@ struct TcLayout {
   static constexpr int OFF_STASH = OFF_BUF + BUFBYTES;
   static constexpr int OFF_BAR = OFF_STASH + STASHBYTES;
   // S ring depth in TMEM: the threshold pass has no O accumulator, so it
-  // keeps four S buffers and its normalizer warps can drift three blocks apart
-  static constexpr int NSB = (MODE == TC_TAU) ? 4 : 2;
-  static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 2 * NSB + 1;
+  // keeps three or four S buffers (its normalizer warps can drift that many
+  // blocks apart) and its Q tile: each QK product takes A (Q) from TMEM and
+  // only B (K) from shared memory, which halves the product's shared-memory
+  // reads (with both operands there a 128 x 128 x 16 product reads as many
+  // bytes per cycle as shared memory delivers)
+  static constexpr int NSB = (MODE == TC_TAU) ? (BN >= 128 ? 3 : 4) : 2;
+  static constexpr int NBAR = 1 + 2 * KST + 2 * VST + 2 * NSB + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // epilogue (m, l) exchange between row halves: reuses the Q tile, which
   // every product has finished reading once the last PV has completed
   static constexpr int OFF_XCH = OFF_Q;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
-  // TMEM columns: the S ring (NSB buffers of BN columns), then O
+  // TMEM columns: the S ring (NSB buffers of BN columns), then O (online)
+  // or Q (threshold pass: bf16 pairs, D / 2 columns)
   static constexpr int TM_S = 0;  // S buffer s at column s * BN
   static constexpr int TM_O = 2 * BN;
-  static constexpr int TM_COLS_USED = (MODE == TC_TAU) ? NSB * BN : 2 * BN + NH * DV;
+  static constexpr int TM_Q = NSB * BN;
+  static constexpr int TM_COLS_USED = (MODE == TC_TAU) ? NSB * BN + D / 2 : 2 * BN + NH * DV;
   static constexpr int TM_COLS = TM_COLS_USED <= 32    ? 32
                                  : TM_COLS_USED <= 64  ? 64
                                  : TM_COLS_USED <= 128 ? 128
@@ -304,12 +310,6 @@ __device__ __forceinline__ float reg_row_tau(const float (&w)[N], bool entmax, f
   return t;
 }
 
-// Weight of a support key from its excess x = u - tau > 0 over the
-// threshold: x for sparsemax, x^2 for 1.5-entmax.
-__device__ __forceinline__ float entmax_weight(float x, const Problem& P) {
-  return P.norm == NATTN_ENTMAX15 ? x * x : x;
-}
-
 // Keep the entries above `lb` (threshold units), compacted in place to the
 // front of the row; returns the new count and, in *kept_sum, the sum of the
 // kept stored values.
@@ -377,6 +377,8 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
   auto bar_sfull = [&](int s) { return smem_addr(&bars[1 + 2 * KST + 2 * VST + s]); };
   auto bar_pfull = [&](int s) { return smem_addr(&bars[1 + 2 * KST + 2 * VST + NSB + s]); };
   const uint32_t bar_pv = smem_addr(&bars[1 + 2 * KST + 2 * VST + 2 * NSB]);
+  // threshold pass: Q has been copied into TMEM (one arrival per normalizer warp)
+  const uint32_t bar_qtm = smem_addr(&bars[2 + 2 * KST + 2 * VST + 2 * NSB]);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + LY::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
 
@@ -395,6 +397,7 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
       mbar_init(bar_pfull(s), NWN);
     }
     mbar_init(bar_pv, 1);
+    mbar_init(bar_qtm, NWN);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -446,7 +449,7 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
       constexpr uint32_t IDESC_S = idesc_bf16(TC_BM, BN, 0, 0);
       constexpr uint32_t IDESC_O = idesc_bf16(TC_BM, DV, 0, 1);
       const uint32_t qbase = smem_addr(smem + LY::OFF_Q);
-      bool ok = mbar_wait_spin(bar_q, 0, abort_flag);
+      bool ok = mbar_wait_spin(MODE == TC_TAU ? bar_qtm : bar_q, 0, abort_flag);
       tc_fence_after();
       for (int j = 0; ok && j <= nseq; ++j) {
         if (j < nseq) {
@@ -466,11 +469,16 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
           const uint32_t sdst = tmem + LY::TM_S + sb * BN;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ad =
-                sdesc_sw128(qbase + (kk >> 2) * TC_BM * 128 + (kk & 3) * 32, 16, 1024);
             const uint64_t bd =
                 sdesc_sw128(kbase + (kk >> 2) * BN * 128 + (kk & 3) * 32, 16, 1024);
-            umma_ss(sdst, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+            if constexpr (MODE == TC_TAU) {
+              // A: dimensions [16 kk, 16 kk + 16) of Q, eight columns in TMEM
+              umma_ts(sdst, tmem + LY::TM_Q + kk * 8, bd, IDESC_S, kk > 0 ? 1u : 0u);
+            } else {
+              const uint64_t ad =
+                  sdesc_sw128(qbase + (kk >> 2) * TC_BM * 128 + (kk & 3) * 32, 16, 1024);
+              umma_ss(sdst, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+            }
           }
           umma_commit(bar_sfull(sb));
           umma_commit(bar_kempty(ks));
@@ -704,9 +712,42 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
         release(j);
       }
     } else {
+      // Q into TMEM: each thread its row's share of the head dimensions, read
+      // from the 128-byte-swizzled tile the TMA left in shared memory (16-byte
+      // chunk c of row r sits at chunk c ^ (r % 8)); column k holds
+      // dimensions 2k (low half) and 2k + 1, the layout of an A operand
+      if (nblk > 0) {
+        alive = mbar_wait(bar_q, 0, abort_flag);
+        constexpr int DH = D / NH;              // dimensions per thread
+        constexpr int PD = DH < 64 ? DH : 64;   // per TMEM store
+#pragma unroll
+        for (int p0 = 0; p0 < DH; p0 += PD) {
+          const int dim0 = half * DH + p0;
+          const uint8_t* qrow = smem + LY::OFF_Q + (dim0 / 64) * TC_BM * 128 + row * 128;
+          uint32_t w[PD / 2];
+#pragma unroll
+          for (int c = 0; c < PD / 8; ++c) {
+            const int cc = (dim0 % 64) / 8 + c;
+            const uint4 x = *reinterpret_cast<const uint4*>(qrow + ((cc ^ (row & 7)) * 16));
+            w[4 * c] = x.x;
+            w[4 * c + 1] = x.y;
+            w[4 * c + 2] = x.z;
+            w[4 * c + 3] = x.w;
+          }
+          if constexpr (PD == 64)
+            tmem_st32(lane_base + LY::TM_Q + dim0 / 2, w);
+          else
+            tmem_st16(lane_base + LY::TM_Q + dim0 / 2, w);
+        }
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_qtm);
+      alive = __all_sync(0xffffffffu, alive);
       // bound pass: bucket maxima
       int kbc = kfirst;
-      for (int j = 0; j < nblk; ++j, kbc = next_kept<BN>(P, b, h, h, qt, kbc + 1, kend)) {
+      for (int j = 0; alive && j < nblk; ++j, kbc = next_kept<BN>(P, b, h, h, qt, kbc + 1, kend)) {
         uint32_t r[64];
         if (!load_scores(j, kbc, r)) {
           alive = false;
@@ -950,51 +991,65 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
 }
 
 
-// Sparse phase 2: one warp per query row.  The row's candidates (every key
-// above a lower bound of its threshold, written by the threshold pass) give
-// the exact threshold by the Newton iteration of thread_row_tau, with the
-// sums taken across the warp; then O = sum over the support of p_j V_j in
-// fp32 on CUDA cores.  The support of sparsemax / 1.5-entmax is a handful of
-// keys per row, so this reads |support| value rows instead of multiplying
-// every block, and the weights enter the sum in full precision.  Lane l
-// owns output columns [l * dv/32, (l+1) * dv/32).
+// Sparse phase 2: RPW query rows per warp (32 / RPW lanes each).  A row's
+// candidates (every key above a lower bound of its threshold, written by the
+// threshold pass) give the exact threshold by the Newton iteration of
+// thread_row_tau, with the sums taken across the row's lanes; then
+// O = sum over the support of p_j V_j in fp32 on CUDA cores.  The support of
+// sparsemax / 1.5-entmax is a handful of keys per row, so this reads
+// |support| value rows instead of multiplying every block, and the weights
+// enter the sum in full precision.  The kernel is bound by latency: with
+// short supports (sparsemax) by its dependent steps, so two rows per warp
+// share them; with longer ones (1.5-entmax) by the value-row loads in
+// flight, which the registers of one row per warp hold more of.  Lane l of a
+// row owns output columns [l * PER, (l+1) * PER).
 constexpr int APPLY_WARPS = 4;
 
-template <int DV, int NSEG, int CAPR>
+template <int DV, int NSEG, int CAPR, int RPW>
 __global__ void __launch_bounds__(APPLY_WARPS * 32)
     sparse_apply_kernel(Problem P, const int* __restrict__ sup_count,
                         const int2* __restrict__ sup_list, const float* __restrict__ rmax,
                         const float* __restrict__ rlb) {
-  constexpr int PER = DV / 32;                  // columns per lane (2, 4 or 8)
+  constexpr int LPR = 32 / RPW;                 // lanes per row
+  constexpr int PER = DV / LPR;                 // columns per lane (2 .. 16)
   constexpr int NCAND = NSEG * CAPR;            // candidates a row can have
-  constexpr int NE = (NCAND + 31) / 32;         // candidate slots per lane
-  __shared__ int2 sup[APPLY_WARPS][NCAND];      // (value row, weight) of the support
+  constexpr int NE = (NCAND + LPR - 1) / LPR;   // candidate slots per lane
+  constexpr int G = 8 / RPW;                    // value rows per gather step
+  constexpr unsigned RMASK = (LPR == 32) ? 0xffffffffu : ((1u << LPR) - 1u);
+  __shared__ int2 sup[APPLY_WARPS][RPW][NCAND];  // (value row, weight) of the support
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int hw = lane / LPR, hl = lane % LPR;   // row of the warp, lane of the row
   const size_t rows =
       P.cu_q != nullptr ? (size_t)P.total_q * P.Hq : (size_t)P.B * P.Hq * P.Tq;
-  const size_t flat = (size_t)blockIdx.x * APPLY_WARPS + wid;
-  if (flat >= rows) return;
   // packed: rows past the last sequence belong to no sequence
-  if (P.cu_q != nullptr && flat >= (size_t)min(P.cu_q[P.B], P.total_q) * P.Hq) return;
+  const size_t owned =
+      P.cu_q != nullptr ? min(rows, (size_t)min(P.cu_q[P.B], P.total_q) * P.Hq) : rows;
+  const size_t row0 = ((size_t)blockIdx.x * APPLY_WARPS + wid) * RPW;
+  if (row0 >= owned) return;  // every row of the warp idle
+  const size_t flat = row0 + hw;
+  // a row that is not there, or that overflowed (the row-wise pass writes
+  // it), still takes part in the warp's shuffles with no candidates
+  const bool there = flat < owned;
   int c[NSEG];
   bool ovf = false;
+  int ntot = 0;
 #pragma unroll
   for (int sg = 0; sg < NSEG; ++sg) {
-    c[sg] = sup_count[flat * NSEG + sg];
+    c[sg] = there ? sup_count[flat * NSEG + sg] : 0;
     ovf |= c[sg] < 0;
-    c[sg] = min(c[sg], CAPR);
   }
-  if (ovf) return;  // the row-wise pass writes this row
-  // slot r of lane l holds entry r * 32 + l of the concatenated segments
+#pragma unroll
+  for (int sg = 0; sg < NSEG; ++sg) {
+    c[sg] = ovf ? 0 : min(c[sg], CAPR);
+    ntot += c[sg];
+  }
+  // slot r of lane l holds entry r * LPR + l of the concatenated segments
   const int2* lst = sup_list + flat * NCAND;
   float w[NE];
   int vr[NE];
-  int ntot = 0;
-#pragma unroll
-  for (int sg = 0; sg < NSEG; ++sg) ntot += c[sg];
 #pragma unroll
   for (int r = 0; r < NE; ++r) {
-    const int e = r * 32 + lane;
+    const int e = r * LPR + hl;
     int at = -1;
     if (e < c[0]) {
       at = e;
@@ -1005,115 +1060,130 @@ __global__ void __launch_bounds__(APPLY_WARPS * 32)
     vr[r] = x.x;
     w[r] = __int_as_float(x.y);
   }
-  float tau = INFINITY;  // less the row maximum
-  if (ntot > 0) {
-    const bool entmax = P.norm == NATTN_ENTMAX15;
-    float t = fmaxf(rlb[flat], -1.f);
-    for (int it = 0; it < 64; ++it) {
-      float cnt = 0.f, s1 = 0.f, s2 = 0.f, wmin = INFINITY;
+  const bool entmax = P.norm == NATTN_ENTMAX15;
+  float t = (ntot > 0) ? fmaxf(rlb[flat], -1.f) : INFINITY;  // less the row maximum
+  // the rows of the warp iterate until all have converged
+  bool done = ntot == 0;
+  for (int it = 0; it < 64 && !__all_sync(0xffffffffu, done); ++it) {
+    float cnt = 0.f, s1 = 0.f, s2 = 0.f, wmin = INFINITY;
 #pragma unroll
-      for (int r = 0; r < NE; ++r) {
-        if (w[r] > t) {
-          cnt += 1.f;
-          s1 += w[r];
-          s2 = fmaf(w[r], w[r], s2);
-          wmin = fminf(wmin, w[r]);
-        }
+    for (int r = 0; r < NE; ++r) {
+      if (w[r] > t) {
+        cnt += 1.f;
+        s1 += w[r];
+        s2 = fmaf(w[r], w[r], s2);
+        wmin = fminf(wmin, w[r]);
       }
-      // xor butterflies: every lane ends with the same sums
+    }
+    // xor butterflies inside the lanes of the row: every lane of the row
+    // ends with the same sums
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-        s1 += __shfl_xor_sync(0xffffffffu, s1, off);
-        s2 += __shfl_xor_sync(0xffffffffu, s2, off);
-        wmin = fminf(wmin, __shfl_xor_sync(0xffffffffu, wmin, off));
-      }
-      float ts, tn;
-      bool valid = true;
-      if (!entmax) {
-        ts = (s1 - 1.f) / cnt;
-        tn = ts;
-      } else {
-        const float mu = s1 / cnt;
-        const float delta = (1.f - (s2 - s1 * mu)) / cnt;
-        valid = delta >= 0.f;
-        ts = valid ? mu - sqrtf(delta) : -INFINITY;
-        const float gv = s2 - 2.f * t * s1 + t * t * cnt;
-        const float gp = 2.f * (s1 - t * cnt);
-        tn = t + (gv - 1.f) / gp;
-      }
-      if (valid && ts >= t && wmin > ts) {
-        t = ts;
-        break;
-      }
-      if (!(tn > t)) break;
+    for (int off = LPR / 2; off > 0; off >>= 1) {
+      cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+      s1 += __shfl_xor_sync(0xffffffffu, s1, off);
+      s2 += __shfl_xor_sync(0xffffffffu, s2, off);
+      wmin = fminf(wmin, __shfl_xor_sync(0xffffffffu, wmin, off));
+    }
+    if (done) continue;
+    float ts, tn;
+    bool valid = true;
+    if (!entmax) {
+      ts = (s1 - 1.f) / cnt;
+      tn = ts;
+    } else {
+      const float mu = s1 / cnt;
+      const float delta = (1.f - (s2 - s1 * mu)) / cnt;
+      valid = delta >= 0.f;
+      ts = valid ? mu - sqrtf(delta) : -INFINITY;
+      const float gv = s2 - 2.f * t * s1 + t * t * cnt;
+      const float gp = 2.f * (s1 - t * cnt);
+      tn = t + (gv - 1.f) / gp;
+    }
+    if (valid && ts >= t && wmin > ts) {
+      t = ts;
+      done = true;
+    } else if (!(tn > t)) {
+      done = true;
+    } else {
       t = tn;
     }
-    tau = t;
   }
-  // the support, compacted in candidate order into this warp's list
+  const float tau = t;
+  // the support, compacted in candidate order into this row's list
   int nsup = 0;
-  const unsigned lt = (1u << lane) - 1u;
+  const unsigned lt = (1u << hl) - 1u;
 #pragma unroll
   for (int r = 0; r < NE; ++r) {
     const float x = w[r] - tau;
     const bool in = x > 0.f;
-    const unsigned bal = __ballot_sync(0xffffffffu, in);
+    const unsigned bal = (__ballot_sync(0xffffffffu, in) >> (LPR * hw)) & RMASK;
     if (in)
-      sup[wid][nsup + __popc(bal & lt)] = make_int2(vr[r], __float_as_int(entmax_weight(x, P)));
+      sup[wid][hw][nsup + __popc(bal & lt)] =
+          make_int2(vr[r], __float_as_int(entmax ? x * x : x));
     nsup += __popc(bal);
   }
   __syncwarp();
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  const bf16* vbase = P.v + lane * PER;
-  auto fma_row = [&](float p, const bf16* vr_) {
-    if constexpr (PER == 8) {
-      const uint4 x = *reinterpret_cast<const uint4*>(vr_);
-      acc[0] += p * bf16lo(x.x); acc[1] += p * bf16hi(x.x);
-      acc[2] += p * bf16lo(x.y); acc[3] += p * bf16hi(x.y);
-      acc[4] += p * bf16lo(x.z); acc[5] += p * bf16hi(x.z);
-      acc[6] += p * bf16lo(x.w); acc[7] += p * bf16hi(x.w);
-    } else if constexpr (PER == 4) {
-      const uint2 x = *reinterpret_cast<const uint2*>(vr_);
-      acc[0] += p * bf16lo(x.x); acc[1] += p * bf16hi(x.x);
-      acc[2] += p * bf16lo(x.y); acc[3] += p * bf16hi(x.y);
+  const bf16* vbase = P.v + hl * PER;
+  // one value row's slice of this lane: PER bf16 in PER / 2 words
+  constexpr int NW = PER / 2;
+  auto load_row = [&](const bf16* vr_, uint32_t (&x)[NW]) {
+    if constexpr (NW >= 4) {
+#pragma unroll
+      for (int q = 0; q < NW / 4; ++q) {
+        const uint4 v = reinterpret_cast<const uint4*>(vr_)[q];
+        x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
+      }
+    } else if constexpr (NW == 2) {
+      const uint2 v = *reinterpret_cast<const uint2*>(vr_);
+      x[0] = v.x; x[1] = v.y;
     } else {
-      const uint32_t x = *reinterpret_cast<const uint32_t*>(vr_);
-      acc[0] += p * bf16lo(x); acc[1] += p * bf16hi(x);
+      x[0] = *reinterpret_cast<const uint32_t*>(vr_);
     }
   };
-  // eight value rows per step, their loads issued before any is used
-  int e = 0;
-  for (; e + 8 <= nsup; e += 8) {
-    int2 en[8];
+  // G value rows per step, their loads issued before any is used (each row
+  // of the warp at its own pace: no shuffles from here on)
+  auto fma_row = [&](float p, const uint32_t (&x)[NW]) {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) en[u] = sup[wid][e + u];
-    if constexpr (PER == 4) {
-      uint2 x[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = *reinterpret_cast<const uint2*>(vbase + (size_t)en[u].x * DV);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float p = __int_as_float(en[u].y);
-        acc[0] += p * bf16lo(x[u].x); acc[1] += p * bf16hi(x[u].x);
-        acc[2] += p * bf16lo(x[u].y); acc[3] += p * bf16hi(x[u].y);
-      }
-    } else {
-#pragma unroll
-      for (int u = 0; u < 8; ++u) fma_row(__int_as_float(en[u].y), vbase + (size_t)en[u].x * DV);
+    for (int k = 0; k < NW; ++k) {
+      acc[2 * k] += p * bf16lo(x[k]);
+      acc[2 * k + 1] += p * bf16hi(x[k]);
     }
+  };
+  int e = 0;
+  for (; e + G <= nsup; e += G) {
+    int2 en[G];
+    uint32_t x[G][NW];
+#pragma unroll
+    for (int u = 0; u < G; ++u) en[u] = sup[wid][hw][e + u];
+#pragma unroll
+    for (int u = 0; u < G; ++u) load_row(vbase + (size_t)en[u].x * DV, x[u]);
+#pragma unroll
+    for (int u = 0; u < G; ++u) fma_row(__int_as_float(en[u].y), x[u]);
   }
   for (; e < nsup; ++e) {
-    const int2 en = sup[wid][e];
-    fma_row(__int_as_float(en.y), vbase + (size_t)en.x * DV);
+    const int2 en = sup[wid][hw][e];
+    uint32_t x[NW];
+    load_row(vbase + (size_t)en.x * DV, x);
+    fma_row(__int_as_float(en.y), x);
   }
-  bf16* o = P.out + flat * DV + lane * PER;
+  if (!there || ovf) return;
+  bf16* o = P.out + flat * DV + hl * PER;
+  uint32_t ov[NW];
 #pragma unroll
-  for (int k = 0; k < PER; k += 2)
-    *reinterpret_cast<uint32_t*>(o + k) = pack_bf16(acc[k], acc[k + 1]);
-  if (lane == 0) {
+  for (int k = 0; k < NW; ++k) ov[k] = pack_bf16(acc[2 * k], acc[2 * k + 1]);
+  if constexpr (NW >= 4) {
+#pragma unroll
+    for (int q = 0; q < NW / 4; ++q)
+      reinterpret_cast<uint4*>(o)[q] = make_uint4(ov[4 * q], ov[4 * q + 1], ov[4 * q + 2], ov[4 * q + 3]);
+  } else if constexpr (NW == 2) {
+    *reinterpret_cast<uint2*>(o) = make_uint2(ov[0], ov[1]);
+  } else {
+    *reinterpret_cast<uint32_t*>(o) = ov[0];
+  }
+  if (hl == 0) {
     if (P.row_stat) P.row_stat[flat] = (ntot > 0) ? rmax[flat] + tau : INFINITY;
     if (P.row_nnz) P.row_nnz[flat] = nsup;
   }

@@ -78,6 +78,13 @@ WORKLOADS = {
                                   128, 128, causal=True, seed=1003,
                                   q_gain=4.0,
                                   normalizers=("sparsemax", "entmax15")),
+    # the same at a quarter of the query scale: flat score rows and wide
+    # supports (about 200 keys per row for 1.5-entmax, against about 23 at
+    # Q x1), beyond the threshold pass's candidate buffers
+    "sparse_prefill_wide": Workload("sparse_prefill_wide", 1, 16, 8, 8192, 8192,
+                                    128, 128, causal=True, seed=1003,
+                                    q_gain=0.25,
+                                    normalizers=("sparsemax", "entmax15")),
     # Gemma-2-9B-shaped local (window 4096) and global layers, soft-cap 50
     "gemma2_9b_local": Workload("gemma2_9b_local", 1, 16, 8, 8192, 8192, 256,
                                 256, causal=True, window=4096, softcap=50.0,
