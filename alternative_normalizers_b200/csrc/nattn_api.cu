@@ -17,6 +17,7 @@
 #include "decode.cuh"
 #include "prefill_pair.cuh"
 #include "prefill_tc.cuh"
+#include "prefill_wide.cuh"
 #include "problem.cuh"
 #include "rowwise.cuh"
 
@@ -155,7 +156,7 @@ struct Plan {
   int R = 0, nsplit = 0, pps = 0;
   // scratch offsets (bytes)
   size_t off_tau = 0, off_ovfc = 0, off_ovfr = 0, off_slots = 0;
-  size_t off_supc = 0, off_supl = 0, off_rlb = 0;
+  size_t off_supc = 0, off_supl = 0, off_rlb = 0, off_wide = 0;
   int sup_cap = 0;
   size_t off_opart = 0, off_ml = 0, off_scores = 0, off_pmask = 0;
   int pm_words = 0;
@@ -170,6 +171,11 @@ bool is_packed(const nattn_args* a) { return a->cu_seqlens_q != nullptr; }
 // Query rows of the problem: B * Hq * Tq, or total_q * Hq when packed.
 long long num_rows(const nattn_args* a) {
   return is_packed(a) ? (long long)a->total_q * a->Hq : (long long)a->B * a->Hq * a->Tq;
+}
+
+// 128-row query tiles of the single-head tensor-core kernels' grid.
+long long ntiles_tc(const nattn_args* a) {
+  return (long long)a->B * a->Hq * ((a->Tq + TC_BM - 1) / TC_BM);
 }
 
 int validate(const nattn_args* a) {
@@ -274,6 +280,9 @@ Plan make_plan(const nattn_args* a) {
       off = up256(off + rows * 2 * 4);
       pl.off_rlb = off;
       off = up256(off + rows * 4);
+      // wide-kernel tile list: its count, then one entry per tile
+      pl.off_wide = off;
+      off = up256(off + 4 + (size_t)ntiles_tc(a) * 4);
       pl.off_supl = off;
       off = up256(off + rows * (size_t)pl.sup_cap * 8);
       pl.row_grid = 2 * 148;
@@ -393,6 +402,7 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
     A.sup_list = nullptr;
     A.sup_cap = 0;
     A.rlb = nullptr;
+    A.wide_tiles = A.wide_count = nullptr;
     // two query heads of one KV group per CTA, each with its own S and O
     if constexpr (D <= 128) {
       if ((a->Hq / a->Hkv) % 2 == 0) {
@@ -437,8 +447,11 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
   A.sup_count = reinterpret_cast<int*>(ws + pl.off_supc);
   A.sup_list = reinterpret_cast<int2*>(ws + pl.off_supl);
   A.rlb = reinterpret_cast<float*>(ws + pl.off_rlb);
+  A.wide_count = reinterpret_cast<int*>(ws + pl.off_wide);
+  A.wide_tiles = A.wide_count + 1;
   A.sup_cap = pl.sup_cap;
   if (cudaMemsetAsync(A.ovf_count, 0, sizeof(int), st) != cudaSuccess) return NATTN_ECUDA;
+  if (cudaMemsetAsync(A.wide_count, 0, sizeof(int), st) != cudaSuccess) return NATTN_ECUDA;
   // d <= 128: each S row split between two warps (eight normalizer warps
   // hide each other's latency); d = 256 keeps whole rows (64-key blocks
   // leave 32 columns per half)
@@ -473,7 +486,20 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
     }
     if (check_launch() != NATTN_OK) return NATTN_ECUDA;
   }
-  // rows whose candidate buffer overflowed: exact row-wise recomputation
+  {
+    // tiles with rows whose candidates overflowed: Newton passes over their
+    // full score rows and a tensor-core weight pass (one CTA per SM walks
+    // the listed tiles; with none listed every CTA exits at once)
+    constexpr int NHW = (2 * BN + 2 * D <= 512) ? 2 : 1;
+    static_assert(NHW == NHT, "the wide kernel reads the threshold pass's row halves");
+    using WL = WideLayout<D, BN, NHW>;
+    auto kw = prefill_wide_kernel<D, BN, NHW>;
+    if (allow_smem(kw, WL::ALLOC) != cudaSuccess) return NATTN_ECUDA;
+    const unsigned wgrid = grid < (unsigned)num_sms() ? grid : (unsigned)num_sms();
+    kw<<<wgrid, WL::THREADS, WL::ALLOC, st>>>(mq, mk, mv, A);
+    if (check_launch() != NATTN_OK) return NATTN_ECUDA;
+  }
+  // rows the wide kernel left unsolved: exact row-wise recomputation
   float* slots = pl.row_slots ? reinterpret_cast<float*>(ws + pl.off_slots) : nullptr;
   return launch_rowwise(P, pl, A.ovf_rows, A.ovf_count, 0, slots, pl.row_grid, st);
 }

@@ -71,6 +71,8 @@ struct TcArgs {
   int2* sup_list;    // TAU: [rows][halves][sup_cap / halves] (value row of the key,
                      //      value less the row maximum in threshold units)
   float* rlb;        // TAU: [rows] lower bound of the threshold less the row maximum
+  int* wide_tiles;   // TAU: tiles (ranks) with a row whose candidates overflowed
+  int* wide_count;   // TAU: number of such tiles (zeroed before the launch)
   int sup_cap;
 };
 
@@ -208,66 +210,9 @@ __device__ __forceinline__ float tc_z(float s, const TcArgs& A) {
   return s * A.zscale;
 }
 
-// Exact threshold of one row's candidate buffer, computed by the thread that
-// owns the row (the 32 rows of a warp are solved side by side).  Stored
-// values are raw scores on the fast path (threshold units = raw * vscale) and
-// threshold units otherwise (vscale = 1); `m` is the row maximum and `t0` a
-// lower bound of tau in shifted units (u - m).
-//
-// Newton's method from the left on g(t) = sum relu(u - t)^k - 1 (k = 1 for
-// sparsemax, 2 for 1.5-entmax), which is convex and decreasing, so every
-// iterate stays at or below the root and {u > t} always contains the
-// support.  At each iterate the closed-form threshold of that set is tried
-// first and accepted once it satisfies the optimality conditions (all members
-// above it, everything else at or below it); for sparsemax this is Michelot's
-// projection algorithm.
-// With max_it below the iteration count to convergence the result is the
-// last Newton iterate: not the threshold, but still a lower bound of it.
-__device__ __forceinline__ float thread_row_tau(const int2* row0, int n0, const int2* row1,
-                                                int n1, float vscale, float m, bool entmax,
-                                                float t0, int max_it = 64) {
-  float t = fmaxf(t0, -1.f);
-  for (int it = 0; it < max_it; ++it) {
-    float cnt = 0.f, s1 = 0.f, s2 = 0.f, wmin = INFINITY;
-    auto add = [&](const int2* row, int n) {
-#pragma unroll 4
-      for (int i = 0; i < n; ++i) {
-        const float w = __int_as_float(row[i].y) * vscale - m;
-        if (w > t) {
-          cnt += 1.f;
-          s1 += w;
-          s2 = fmaf(w, w, s2);
-          wmin = fminf(wmin, w);
-        }
-      }
-    };
-    add(row0, n0);
-    add(row1, n1);
-    float ts, tn;
-    bool valid = true;
-    if (!entmax) {
-      ts = (s1 - 1.f) / cnt;
-      tn = ts;
-    } else {
-      const float mu = s1 / cnt;
-      const float delta = (1.f - (s2 - s1 * mu)) / cnt;
-      valid = delta >= 0.f;
-      ts = valid ? mu - sqrtf(delta) : -INFINITY;
-      const float g = s2 - 2.f * t * s1 + t * t * cnt;
-      const float gp = 2.f * (s1 - t * cnt);
-      tn = t + (g - 1.f) / gp;
-    }
-    if (valid && ts >= t && wmin > ts) return ts + m;
-    if (!(tn > t)) break;
-    t = tn;
-  }
-  return t + m;
-}
-
-// Exact threshold of N values held in registers, in shifted threshold units
-// (w = u - m with m the row maximum; -inf for no key), by the Newton
-// iteration of thread_row_tau: every iterate is a lower bound of the
-// threshold.  Returns it in shifted units.
+// Exact threshold of N values held in registers (shifted threshold units;
+// -inf for no key) by tau_step from t0: every iterate is a lower bound of
+// the threshold.  Returns it in shifted units.
 template <int N>
 __device__ __forceinline__ float reg_row_tau(const float (&w)[N], bool entmax, float t0,
                                              int max_it = 32) {
@@ -288,45 +233,9 @@ __device__ __forceinline__ float reg_row_tau(const float (&w)[N], bool entmax, f
       q1 = fmaf(x1, x1, q1);
       wmin = fminf(wmin, fminf(in0 ? w[i] : INFINITY, in1 ? w[i + 1] : INFINITY));
     }
-    const float cnt = c0 + c1, s1 = a0 + a1, s2 = q0 + q1;
-    float ts, tn;
-    bool valid = true;
-    if (!entmax) {
-      ts = (s1 - 1.f) / cnt;
-      tn = ts;
-    } else {
-      const float mu = s1 / cnt;
-      const float delta = (1.f - (s2 - s1 * mu)) / cnt;
-      valid = delta >= 0.f;
-      ts = valid ? mu - sqrtf(delta) : -INFINITY;
-      const float g = s2 - 2.f * t * s1 + t * t * cnt;
-      const float gp = 2.f * (s1 - t * cnt);
-      tn = t + (g - 1.f) / gp;
-    }
-    if (valid && ts >= t && wmin > ts) return ts;
-    if (!(tn > t)) break;
-    t = tn;
+    if (tau_step(c0 + c1, a0 + a1, q0 + q1, wmin, entmax, t) != 0) break;
   }
   return t;
-}
-
-// Keep the entries above `lb` (threshold units), compacted in place to the
-// front of the row; returns the new count and, in *kept_sum, the sum of the
-// kept stored values.
-__device__ __forceinline__ int thread_compact_row(int2* row, int n, float vscale, float lb,
-                                                  float* kept_sum) {
-  int j = 0;
-  float sum = 0.f;
-  for (int i = 0; i < n; ++i) {
-    const int2 e = row[i];
-    const float v = __int_as_float(e.y);
-    if (v * vscale > lb) {
-      row[j++] = e;
-      sum += v;
-    }
-  }
-  *kept_sum = sum;
-  return j;
 }
 
 template <int D, int DV, int BN, int KST, int VST, int MODE, int NH = 1>
@@ -399,6 +308,7 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
     mbar_init(bar_pv, 1);
     mbar_init(bar_qtm, NWN);
     *abort_flag = 0;
+    misc[2] = 0;  // threshold pass: some row of the tile overflowed
     fence_barrier_init();
   }
   if (warp == NWN + 1) {
@@ -832,30 +742,13 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
             }
             nbuf += na;
           };
-          // when a row's buffer cannot take this chunk's candidates (a support
-          // far wider than the bucket set), every row of the warp raises its
-          // bound by one Newton step towards the threshold of the keys it has
-          // kept and compacts (each thread its own row, side by side); if the
-          // candidates still do not fit, the exact threshold is taken with them
-          // included, a few rounds at most, and only then is the row listed
-          // for the row-wise pass
-          if (__any_sync(0xffffffffu, nbuf + __popc(msk) > LY::CAPR)) {
-            float ksum;
-            lb = fmaxf(lb, thread_row_tau(mybuf, nbuf, mybuf, 0, vs, m_run, entmax, lb - m_run, 1));
-            nbuf = thread_compact_row(mybuf, nbuf, vs, lb, &ksum);
-            thr = to_thr(lb);
-            msk &= cand_mask(thr);
-            for (int round = 0; round < 4 && nbuf + __popc(msk) > LY::CAPR; ++round) {
-              append(LY::CAPR - nbuf);
-              lb = fmaxf(lb, thread_row_tau(mybuf, nbuf, mybuf, 0, vs, m_run, entmax, lb - m_run));
-              nbuf = thread_compact_row(mybuf, nbuf, vs, lb, &ksum);
-              thr = to_thr(lb);
-              msk &= cand_mask(thr);
-            }
-            if (nbuf + __popc(msk) > LY::CAPR) {
-              ovf = true;
-              msk = 0;
-            }
+          // a row whose buffer cannot take this chunk's candidates has a
+          // support far wider than the buffer (with the bucket bound the
+          // candidates are the support and about one key more): it stops
+          // collecting, and the wide kernel takes its tile
+          if (nbuf + __popc(msk) > LY::CAPR) {
+            ovf = true;
+            msk = 0;
           }
           if (__any_sync(0xffffffffu, msk != 0)) append(32);
         }
@@ -870,7 +763,7 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
       // the key, value less the row maximum in threshold units); the apply
       // kernel solves every row's exact threshold with a warp per row and
       // gathers its support.  A row whose candidates overflowed in either
-      // half is listed for the row-wise pass instead.
+      // half is marked (count -1) and its tile listed for the wide kernel.
       bool ovf_r = ovf;
       float lb_r = lb;
       if constexpr (NH > 1) {
@@ -884,11 +777,8 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
       if (row_ok) {
         const size_t seg = flat * NH + half;
         if (ovf_r) {
-          if (half == 0) {
-            const int slot = atomicAdd(A.ovf_count, 1);
-            A.ovf_rows[slot] = (int)flat;
-          }
           A.sup_count[seg] = -1;
+          if (half == 0) atomicOr(&misc[2], 1u);
         } else {
           int2* dst = A.sup_list + seg * LY::CAPR;
           for (int i = 0; i < nbuf; ++i) {
@@ -988,13 +878,16 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
   __syncthreads();
   tc_fence_after();
   if (warp == NWN + 1) tmem_dealloc(tmem, LY::TM_COLS);
+  if constexpr (MODE == TC_TAU) {
+    if (tid == 0 && misc[2] != 0) A.wide_tiles[atomicAdd(A.wide_count, 1)] = rank;
+  }
 }
 
 
 // Sparse phase 2: RPW query rows per warp (32 / RPW lanes each).  A row's
 // candidates (every key above a lower bound of its threshold, written by the
 // threshold pass) give the exact threshold by the Newton iteration of
-// thread_row_tau, with the sums taken across the row's lanes; then
+// tau_step, with the sums taken across the row's lanes; then
 // O = sum over the support of p_j V_j in fp32 on CUDA cores.  The support of
 // sparsemax / 1.5-entmax is a handful of keys per row, so this reads
 // |support| value rows instead of multiplying every block, and the weights
@@ -1085,28 +978,7 @@ __global__ void __launch_bounds__(APPLY_WARPS * 32)
       wmin = fminf(wmin, __shfl_xor_sync(0xffffffffu, wmin, off));
     }
     if (done) continue;
-    float ts, tn;
-    bool valid = true;
-    if (!entmax) {
-      ts = (s1 - 1.f) / cnt;
-      tn = ts;
-    } else {
-      const float mu = s1 / cnt;
-      const float delta = (1.f - (s2 - s1 * mu)) / cnt;
-      valid = delta >= 0.f;
-      ts = valid ? mu - sqrtf(delta) : -INFINITY;
-      const float gv = s2 - 2.f * t * s1 + t * t * cnt;
-      const float gp = 2.f * (s1 - t * cnt);
-      tn = t + (gv - 1.f) / gp;
-    }
-    if (valid && ts >= t && wmin > ts) {
-      t = ts;
-      done = true;
-    } else if (!(tn > t)) {
-      done = true;
-    } else {
-      t = tn;
-    }
+    done = tau_step(cnt, s1, s2, wmin, entmax, t) != 0;
   }
   const float tau = t;
   // the support, compacted in candidate order into this row's list

@@ -168,4 +168,40 @@ __device__ __forceinline__ const bf16* key_row(const Problem& P, const bf16* bas
   return base + (((size_t)page * P.Hkv + g) * P.page_size + (j % P.page_size)) * dim;
 }
 
+// One step of the threshold iteration.  With w the scores in threshold units
+// less the row maximum, g(t) = sum relu(w - t)^k - 1 (k = 1 for sparsemax,
+// 2 for 1.5-entmax) is convex and decreasing and its root is tau.  From the
+// count, sum, sum of squares and minimum of the w above the iterate t, the
+// closed-form threshold of that set is accepted once it satisfies the
+// optimality conditions (every member of the set above it; the set holds
+// everything above t, and t stays at or below the root); otherwise Newton's
+// method moves t right, never past the root, so {w > t} always contains the
+// support.  For sparsemax this is Michelot's projection algorithm.  Returns
+// 1 when t is now the threshold, 0 when t moved and another step is needed,
+// -1 when no progress is possible (t stays a lower bound of the threshold).
+__device__ __forceinline__ int tau_step(float cnt, float s1, float s2, float wmin, bool entmax,
+                                        float& t) {
+  float ts, tn;
+  bool valid = true;
+  if (!entmax) {
+    ts = (s1 - 1.f) / cnt;
+    tn = ts;
+  } else {
+    const float mu = s1 / cnt;
+    const float delta = (1.f - (s2 - s1 * mu)) / cnt;
+    valid = delta >= 0.f;
+    ts = valid ? mu - sqrtf(delta) : -INFINITY;
+    const float g = s2 - 2.f * t * s1 + t * t * cnt;
+    const float gp = 2.f * (s1 - t * cnt);
+    tn = t + (g - 1.f) / gp;
+  }
+  if (valid && ts >= t && wmin > ts) {
+    t = ts;
+    return 1;
+  }
+  if (!(tn > t)) return -1;
+  t = tn;
+  return 0;
+}
+
 }  // namespace nattn

@@ -95,27 +95,7 @@ __device__ float block_solve_tau(const float* sc, int n, float m, bool entmax,
       }
     }
     const Red4 r = block_red4(acc, red);
-    const float cnt = r.a, s1 = r.b, s2 = r.c, wmin = r.d;
-    float ts, tn;
-    bool valid = true;
-    if (!entmax) {
-      ts = (s1 - 1.f) / cnt;
-      tn = ts;
-    } else {
-      const float mu = s1 / cnt;
-      const float delta = (1.f - (s2 - s1 * mu)) / cnt;
-      valid = delta >= 0.f;
-      ts = valid ? mu - sqrtf(delta) : -INFINITY;
-      const float g = s2 - 2.f * t * s1 + t * t * cnt;
-      const float gp = 2.f * (s1 - t * cnt);
-      tn = t + (g - 1.f) / gp;
-    }
-    if (valid && ts >= t && wmin > ts) {
-      t = ts;
-      break;
-    }
-    if (!(tn > t)) break;
-    t = tn;
+    if (tau_step(r.a, r.b, r.c, r.d, entmax, t) != 0) break;
   }
   return t + m;
 }

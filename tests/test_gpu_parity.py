@@ -141,6 +141,38 @@ def test_tc_sparse_overflow_rows(normalizer):
     check_stat(st, s)
 
 
+@pytest.mark.parametrize("normalizer,qscale", [("sparsemax", 1 / 128), ("entmax15", 1 / 8)])
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_tc_sparse_wide_supports(normalizer, qscale, d):
+    """Flat score rows (queries scaled down): supports of up to a few
+    hundred keys, wider than the threshold pass's candidate buffers on most
+    rows past the first tile.  Those rows take the wide kernel (Newton
+    passes over their full score rows, weights multiplied on the tensor
+    cores); the first rows of the causal band stay within the buffers, so
+    tiles hold both kinds.  Output, threshold and support size (row_nnz)
+    against the oracle, on a ragged 1000-row causal problem."""
+    import torch
+    import oracle
+    from alternative_normalizers_b200 import attention, nattn_get_device_status
+    T = 1000
+    q, k, v = _inputs(41 + d, 1, 4, 2, T, T, d)
+    q = (q.float() * qscale).to(q.dtype)
+    nnz = torch.full((1, 4, T), -1, dtype=torch.int32, device="cuda")
+    out, st, _ = attention(q.cuda(), k.cuda(), v.cuda(), normalizer=normalizer,
+                           causal=True, row_nnz=nnz)
+    torch.cuda.synchronize()
+    assert nattn_get_device_status() == 0
+    o, s, w = oracle.attention_fwd(q, k, v, d ** -0.5, normalizer, True,
+                                   want_weights=True)
+    want_nnz = (w > 0).sum(axis=-1)
+    # the case exercises what it is meant to: supports beyond the buffers
+    assert want_nnz.max() > 200
+    check_out(out.float().cpu().numpy(), o)
+    check_stat(st.cpu().numpy(), s)
+    diff = np.abs(nnz.cpu().numpy().astype(np.int64) - want_nnz)
+    assert diff.max() <= 1 and (diff == 0).mean() >= 0.99
+
+
 def test_softmax1_is_softmax_with_zero_key_on_gpu():
     """GPU softmax1 equals GPU softmax on the input with a zero key and zero
     value prepended (bottom-right causal), which also exercises Tk' = T + 1."""
