@@ -328,11 +328,17 @@ __global__ void __launch_bounds__((4 * NH + 2) * 32, 1)
       tmem_ld32(saddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
       tmem_ld32(saddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
       tmem_ld_wait();
+      if (fast) {
 #pragma unroll
-      for (int k = 0; k < 64; ++k) {
-        const float x = fast ? fmaf(__uint_as_float(r[k]), A.zscale, -m)
-                             : tc_z(__uint_as_float(r[k]), A) - m;
-        w[k] = (edge && (unsigned)(k - klb) > span) ? -INFINITY : x;
+        for (int k = 0; k < 64; ++k) w[k] = fmaf(__uint_as_float(r[k]), A.zscale, -m);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 64; ++k) w[k] = tc_z(__uint_as_float(r[k]), A) - m;
+      }
+      if (edge) {
+#pragma unroll
+        for (int k = 0; k < 64; ++k)
+          if ((unsigned)(k - klb) > span) w[k] = -INFINITY;
       }
       return true;
     };

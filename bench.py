@@ -702,8 +702,8 @@ def detail(args, dev, flush):
     import torch
     from alternative_normalizers_b200.workloads import WORKLOADS
     res = {}
-    names = ["sparse_prefill_t1", "sparse_prefill_t4", "gemma2_9b_local",
-             "gemma2_9b_global", "paged_decode"]
+    names = ["sparse_prefill_t1", "sparse_prefill_t4", "sparse_prefill_wide",
+             "gemma2_9b_local", "gemma2_9b_global", "paged_decode"]
     for name in names:
         w = WORKLOADS[name]
         try:
