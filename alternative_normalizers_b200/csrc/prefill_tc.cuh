@@ -591,21 +591,23 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
         float s0 = 0.f, s1 = 0.f;
         uint32_t pk[32];  // 64 scores -> 32 packed columns
         exp2_pack64(&r[0], fa, msafe, s0, s1, pk);
-        // P(j) is stored only once the previous block's PV has completed, so
-        // no TMEM store overlaps a product that reads TMEM (that product was
-        // issued a whole block of exponentials earlier: the wait rarely
-        // stalls); this also orders the O rescale below
-        if (j > 0 &&
-            !__all_sync(0xffffffffu, mbar_wait_spin(bar_pv, (j - 1) & 1, abort_flag))) {
-          alive = false;
-          break;
-        }
-        tc_fence_after();
+        // P(j) goes over S(j)'s own columns; the products in flight read or
+        // write the other S buffer and O
         tmem_st32(paddr, pk);
         tmem_st_wait();
         l_run = l_run * alpha + (s0 + s1);
-        // rescale O when the maximum moved (warp-uniform TMEM access)
+        // Rescale O when the maximum moved (warp-uniform TMEM access).  With
+        // two S buffers QK(j) can complete before PV(j-1) is even issued, so
+        // PV(j-1) may still be accumulating into O here: the rescale waits
+        // for it (reading and rewriting O under an in-flight product loses
+        // that product's sum).  PV(j) waits for this block's P, which is
+        // released after the rescale.
         if (__any_sync(0xffffffffu, resc) && j > 0) {
+          if (!__all_sync(0xffffffffu, mbar_wait_spin(bar_pv, (j - 1) & 1, abort_flag))) {
+            alive = false;
+            break;
+          }
+          tc_fence_after();
           const uint32_t oaddr = lane_base + LY::TM_O + half * DV;
 #pragma unroll 1
           for (int c = 0; c < DV / 32; ++c) {

@@ -173,6 +173,33 @@ def test_tc_sparse_wide_supports(normalizer, qscale, d):
     assert diff.max() <= 1 and (diff == 0).mean() >= 0.99
 
 
+@pytest.mark.parametrize("normalizer", ("softmax", "softmax1"))
+@pytest.mark.parametrize("d,Hq", [(256, 2), (128, 3)])
+def test_online_rescale_every_block(normalizer, d, Hq):
+    """Scores that rise by about 9 (log2 units) from one 64-key block to the
+    next: the running maximum moves past the lazy-rescale margin of 8 on
+    every block, so the single-tile kernel (d = 256, and odd GQA groups)
+    rescales O on every block while the previous block's PV may still be in
+    flight.  Each block's keys tie, so the weights of earlier blocks stay
+    visible in O (about 2^-9 per block back)."""
+    import torch
+    import oracle
+    T = 1024
+    g = torch.Generator().manual_seed(77 + d)
+    q = torch.zeros(1, Hq, T, d)
+    q[..., 0] = 4.0
+    k = torch.randn(1, 1, T, d, generator=g) * 0.01
+    # x = q.k * scale * log2(e) rises by ~9 per 64 keys
+    step = 9.0 / (4.0 * d ** -0.5 * 1.4426950408889634)
+    k[0, 0, :, 0] = step * (torch.arange(T) // 64).float()
+    v = torch.randn(1, 1, T, d, generator=g)
+    q, k, v = q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+    out, st, _ = _gpu(q, k, v, normalizer=normalizer, causal=True)
+    o, s, _ = oracle.attention_fwd(q, k, v, d ** -0.5, normalizer, True)
+    check_out(out, o)
+    check_stat(st, s)
+
+
 def test_softmax1_is_softmax_with_zero_key_on_gpu():
     """GPU softmax1 equals GPU softmax on the input with a zero key and zero
     value prepended (bottom-right causal), which also exercises Tk' = T + 1."""
