@@ -188,6 +188,17 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+// Wait for the last two completions of an mbarrier that completes once per
+// block (a PV product's commit): blocks g_last - 1 and g_last.  A parity
+// wait is only meaningful while the barrier is at most one phase behind the
+// awaited one (a phase two back has the same parity and counts as done), so
+// a consumer that may be two products behind waits for both, oldest first.
+__device__ __forceinline__ bool mbar_wait_last2(uint32_t bar, int g_last, bool two,
+                                                volatile int* abort) {
+  if (two && !mbar_wait(bar, (g_last - 1) & 1, abort)) return false;
+  return mbar_wait(bar, g_last & 1, abort);
+}
+
 // Bounded wait that polls with a short sleep between polls instead of asking
 // to be suspended: for waits whose reaction time is on the critical path
 // (the MMA issuer, the normalizer warps), while leaving the issue slots of

@@ -421,11 +421,11 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
                          : prefill_pair_kernel<D, KST, VST, true, false, PAIR_DENSE>)
                    : (bm ? prefill_pair_kernel<D, KST, VST, false, true, PAIR_DENSE>
                          : prefill_pair_kernel<D, KST, VST, false, false, PAIR_DENSE>);
-        if (allow_smem(kp, PL::ALLOC) != cudaSuccess) return NATTN_ECUDA;
         // persistent: one CTA per SM (shared memory and TMEM allow one), each
         // walking its share of the tiles
         const long long ntiles = (long long)a->B * (a->Hq / 2) * ntq;
         const unsigned pgrid = (unsigned)(ntiles < num_sms() ? ntiles : num_sms());
+        if (allow_smem(kp, PL::ALLOC) != cudaSuccess) return NATTN_ECUDA;
         kp<<<pgrid, PAIR_THREADS, PL::ALLOC, st>>>(mq, mk, mv, A);
         return check_launch();
       }

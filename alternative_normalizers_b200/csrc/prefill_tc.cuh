@@ -796,9 +796,11 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
         }
       }
     } else {
+      // with two S buffers the last two PVs may both be in flight here (S(j)
+      // only guarantees PV(j - 2)): wait for both
       const bool have_o =
           __all_sync(0xffffffffu, alive && nblk > 0 &&
-                                      mbar_wait(bar_pv, (nblk - 1) & 1, abort_flag));
+                                      mbar_wait_last2(bar_pv, nblk - 1, nblk > 1, abort_flag));
       tc_fence_after();
       // combine the halves: scale factors ca (half 0) and cb (half 1)
       float ca = 1.f, cb = 0.f, stat = tau;
