@@ -535,15 +535,44 @@ __global__ void __launch_bounds__(TAU_THREADS)
   for (int w = threadIdx.x; w < A.pm_words; w += TAU_THREADS) smask[w] = 0u;
   __syncthreads();
   const float* zrow = A.scores + (size_t)row * P.Tk;
-  for (int j = threadIdx.x; j < Lk; j += TAU_THREADS) {
-    const float u = zrow[j];
-    if (u > m - 1.f) {
-      const int k = atomicAdd(&s_n, 1);
+  // candidates: one shared atomic per warp and batch of keys (ballot +
+  // population count), four scores per thread per load where the row is
+  // 16-byte aligned
+  const unsigned lt = (1u << (threadIdx.x & 31)) - 1u;
+  auto put = [&](bool in, float u, int j) {
+    const unsigned bal = __ballot_sync(0xffffffffu, in);
+    if (bal == 0u) return;
+    int base = 0;
+    if ((threadIdx.x & 31) == __ffs(bal) - 1) base = atomicAdd(&s_n, __popc(bal));
+    base = __shfl_sync(0xffffffffu, base, __ffs(bal) - 1);
+    if (in) {
+      const int k = base + __popc(bal & lt);
       if (k < cap) {
         cand[k] = u;
         cidx[k] = j;
       }
     }
+  };
+  const float thr = m - 1.f;
+  const bool vec = (reinterpret_cast<uintptr_t>(zrow) & 15u) == 0;
+  const int nvec = vec ? Lk / 4 : 0;
+  // every thread of a warp runs the same number of trips (ballots above)
+  const int trips = (nvec + TAU_THREADS - 1) / TAU_THREADS;
+  for (int t = 0; t < trips; ++t) {
+    const int q = t * TAU_THREADS + threadIdx.x;
+    float4 x = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    if (q < nvec) x = reinterpret_cast<const float4*>(zrow)[q];
+    put(x.x > thr, x.x, 4 * q);
+    put(x.y > thr, x.y, 4 * q + 1);
+    put(x.z > thr, x.z, 4 * q + 2);
+    put(x.w > thr, x.w, 4 * q + 3);
+  }
+  const int rest = Lk - 4 * nvec;
+  const int trips1 = (rest + TAU_THREADS - 1) / TAU_THREADS;
+  for (int t = 0; t < trips1; ++t) {
+    const int j = 4 * nvec + t * TAU_THREADS + threadIdx.x;
+    const float u = (j < Lk) ? zrow[j] : -INFINITY;
+    put(u > thr, u, j);
   }
   __syncthreads();
   const int n = s_n;
