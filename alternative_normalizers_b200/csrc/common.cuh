@@ -221,6 +221,27 @@ __device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity,
   }
 }
 
+// Bounded wait that polls without sleeping: for the hand-offs of the online
+// pair kernel, where every poll's reaction time is on the critical path of
+// a tile and the warps that share the sub-partition are waiting too
+// (measured 0.7 % faster there than polling with a short sleep).
+__device__ __forceinline__ bool mbar_wait_busy(uint32_t bar, uint32_t parity,
+                                               volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 1023u) == 0) {
+      if (abort != nullptr && *abort) return false;
+      if (globaltimer() - t0 > NATTN_WAIT_NS) {
+        set_status(NATTN_ETIMEOUT);
+        if (abort != nullptr) *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // TMA (tensor and plain bulk copies, global -> shared, no multicast)
 // ---------------------------------------------------------------------------

@@ -155,7 +155,7 @@ __device__ __forceinline__ bool prefill_pair_normalizer(
   int nvis = 0;  // visible keys in kept blocks (row_nnz)
 
   for (int j = 0; j < nblk; ++j) {
-    if (!__all_sync(0xffffffffu, mbar_wait_spin(bar_sf, (g0 + j) & 1, abort_flag))) {
+    if (!__all_sync(0xffffffffu, mbar_wait_busy(bar_sf, (g0 + j) & 1, abort_flag))) {
       alive = false;
       break;
     }
@@ -485,11 +485,11 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
         const PairTile T = SORTED ? tile_of(rank) : pair_tile<LAY>(P, rank);
         const int nblk = T.nblk;
         if (nblk == 0) continue;
-        ok = mbar_wait_spin(bar_q, tq & 1, abort_flag);
+        ok = mbar_wait_busy(bar_q, tq & 1, abort_flag);
         tc_fence_after();
         // prologue: both tiles' scores of the first block (S of either tile
         // held the previous tile's last P, whose PV was issued before)
-        if (ok && mbar_wait_spin(bar_kfull(g0 % KST), (g0 / KST) & 1, abort_flag)) {
+        if (ok && mbar_wait_busy(bar_kfull(g0 % KST), (g0 / KST) & 1, abort_flag)) {
           tc_fence_after();
           issue_qk(0, g0);
           issue_qk(1, g0);
@@ -501,13 +501,13 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
         for (int j = 0; ok && j < nblk; ++j) {
           const int gj = g0 + j;
           const int vs = gj % VST;
-          if (!mbar_wait_spin(bar_vfull(vs), (gj / VST) & 1, abort_flag)) {
+          if (!mbar_wait_busy(bar_vfull(vs), (gj / VST) & 1, abort_flag)) {
             ok = false;
             break;
           }
           bool k_next = false;
           for (int t = 0; t < 2; ++t) {
-            if (!mbar_wait_spin(bar_pfull(t), gj & 1, abort_flag)) {
+            if (!mbar_wait_busy(bar_pfull(t), gj & 1, abort_flag)) {
               ok = false;
               break;
             }
@@ -525,7 +525,7 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
             if (j + 1 < nblk) {
               // this tile's next scores go in behind its PV (issue order)
               if (t == 0) {
-                if (!mbar_wait_spin(bar_kfull((gj + 1) % KST), ((gj + 1) / KST) & 1,
+                if (!mbar_wait_busy(bar_kfull((gj + 1) % KST), ((gj + 1) / KST) & 1,
                                     abort_flag)) {
                   ok = false;
                   break;
