@@ -11,16 +11,19 @@
 // The path is bound by HBM bandwidth (4 KiB of K+V per token at Hkv = 8,
 // d = 128), so the design is about the loads: each (page, kv head) slab is
 // contiguous in the pool and is brought into shared memory by TMA in 64-column
-// boxes with the 128-byte swizzle, several pages ahead, one mbarrier per
-// stage.  The arithmetic per page is tiny (16 x 64 x 128 per product) and
-// runs on warp-level mma.sync so that it never competes with the loads for
-// issue slots; row reductions use warp shuffles.
+// boxes with the 128-byte swizzle, one mbarrier per stage.  A CTA's time per
+// page is mostly latency (the page's barrier, the products, the block
+// barriers), so the ring is two stages deep and the bytes in flight come from
+// three to five CTAs per SM.  The arithmetic per page is tiny (16 x 64 x 128
+// per product) and runs on warp-level mma.sync so that it never competes with
+// the loads for issue slots; row reductions use warp shuffles.
 //
 // Modes:
 //   ONLINE  softmax / softmax1: running (max, sum, O) per split in log2 units,
 //           merged by decode_combine_kernel (softmax1 adds its sink once there).
-//   SCORES  sparse pass 1: write every score (in threshold units) and the
-//           split's row maximum to scratch.
+//   SCORES  sparse pass 1: write every score (in threshold units) to scratch
+//           straight from the product's accumulators, and the split's row
+//           maximum.
 //   APPLY   sparse pass 3: given tau per row, skip pages with no weight above
 //           zero (their V is never loaded), accumulate p V for the rest.
 #pragma once
@@ -215,6 +218,23 @@ __global__ void __launch_bounds__(DEC_THREADS)
 #pragma unroll
     for (int e = 0; e < 4; ++e) oacc[n][e] = 0.f;
 
+  // SCORES: each thread's score rows (nt * 8 + 2 * t4 + h) in the scratch,
+  // and their running maxima over the thread's keys
+  float* srow[NTR][2];
+  float mreg[NTR][2];
+#pragma unroll
+  for (int nt = 0; nt < NTR; ++nt)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = nt * 8 + 2 * t4 + h;
+      srow[nt][h] = nullptr;
+      mreg[nt][h] = -INFINITY;
+      if constexpr (MODE == DEC_SCORES)
+        if (r < R)
+          srow[nt][h] = A.scores +
+                        (((size_t)b * P.Hq + g * group + r / P.Tq) * P.Tq + r % P.Tq) * P.Tk;
+    }
+
   // zero the unused P rows once (rows >= R stay zero)
   for (int x = tid; x < (L::OFF_A - L::OFF_P) / 4; x += DEC_THREADS)
     reinterpret_cast<uint32_t*>(Pb)[x] = 0u;
@@ -280,31 +300,20 @@ __global__ void __launch_bounds__(DEC_THREADS)
                 z = P.softcap * fast_tanh(sc / P.softcap) * (A.zscale / P.scale);
               }
               const bool ok = !bad && j >= rr.lo && j <= rr.hi;
-              S[r * L::SSTRIDE + tok] = ok ? z : -INFINITY;
+              if constexpr (MODE == DEC_SCORES) {
+                // straight from the accumulators: 8 lanes cover 8
+                // consecutive keys of a row (32-byte segments)
+                const float zz = ok ? z : -INFINITY;
+                if (j < Lk) srow[nt][e & 1][j] = zz;
+                mreg[nt][e & 1] = fmaxf(mreg[nt][e & 1], zz);
+              } else {
+                S[r * L::SSTRIDE + tok] = ok ? z : -INFINITY;
+              }
             }
           }
         }
       }
-      __syncthreads();
-    }
-
-    if constexpr (MODE == DEC_SCORES) {
-      // write scores (coalesced row segments) and track the row maximum
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int r = warp + 4 * k;
-        if (r >= R) break;
-        const int hh = r / P.Tq, i = r % P.Tq;
-        const size_t row = ((size_t)b * P.Hq + g * group + hh) * P.Tq + i;
-        float mx = -INFINITY;
-        for (int jj = lane; jj < PS; jj += 32) {
-          const int j = j0 + jj;
-          const float z = S[r * L::SSTRIDE + jj];
-          if (j < Lk) A.scores[row * P.Tk + j] = z;
-          mx = fmaxf(mx, z);
-        }
-        m_run[k] = fmaxf(m_run[k], warp_max(mx));
-      }
+      if constexpr (MODE != DEC_SCORES) __syncthreads();
     }
 
     if constexpr (MODE == DEC_ONLINE) {
@@ -401,6 +410,28 @@ __global__ void __launch_bounds__(DEC_THREADS)
     if (tid == 0 && it + NS < count) {
       fence_proxy_async();
       issue(it + NS);
+    }
+  }
+
+  if constexpr (MODE == DEC_SCORES) {
+    // row maxima: over the 8 lanes sharing a row, then over the warps
+    float* smax = S;  // [4 warps][16 rows]
+#pragma unroll
+    for (int nt = 0; nt < NTR; ++nt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float v = mreg[nt][h];
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+        if (gq == 0) smax[warp * 16 + nt * 8 + 2 * t4 + h] = v;
+      }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int r = warp + 4 * k;
+      if (r < R)
+        m_run[k] = fmaxf(fmaxf(smax[r], smax[16 + r]), fmaxf(smax[32 + r], smax[48 + r]));
     }
   }
 

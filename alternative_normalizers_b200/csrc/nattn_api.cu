@@ -507,9 +507,11 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
 template <int D, int PS, int MODE>
 int launch_decode_mode(const nattn_args* a, const DecodeArgs& A, const CUtensorMap& mk,
                        const CUtensorMap& mv, cudaStream_t st) {
-  using L1 = DecodeSmem<D, D, PS, 2, MODE>;
-  // about 100 KB of stages: two CTAs per SM for K+V pages, three for K or V
-  constexpr int NS = (L1::STAGE * 4 <= 100 * 1024) ? 4 : (L1::STAGE * 3 <= 100 * 1024 ? 3 : 2);
+  // two stages (one page computing, the next loading): a CTA's time per page
+  // is mostly its own barrier and product latency, so more CTAs per SM (three
+  // for K+V pages of d = 128, five for K or V alone) move more bytes than
+  // deeper rings do; with four stages the same passes ran 24-32 % slower
+  constexpr int NS = 2;
   using L = DecodeSmem<D, D, PS, NS, MODE>;
   // only the sparse apply pass keeps a page list (two ints per page)
   const int bytes = L::BYTES_NOLIST + (MODE == DEC_APPLY ? 2 * A.pps * 4 : 0) + 1024;

@@ -256,6 +256,32 @@ def test_paged_decode(normalizer, page, d, Tq):
         check_stat(st[b].cpu().numpy(), res[b][1], f"seq {b}")
 
 
+@pytest.mark.parametrize("normalizer", ["sparsemax", "entmax15"])
+@pytest.mark.parametrize("page,gain", [(64, 0.02), (64, 0.3), (32, 0.1)])
+def test_paged_decode_long_and_flat(normalizer, page, gain):
+    """Sequences of several splits and queries scaled down so that scores
+    crowd near their maximum: thousands of threshold candidates per row (more
+    than the threshold kernel keeps in shared memory at the smallest gain)
+    and supports longer than the apply pass's per-split list."""
+    import torch
+    import oracle
+    from alternative_normalizers_b200 import paged_attention
+    from alternative_normalizers_b200 import nattn_get_device_status
+    B, Hq, Hkv, d = 3, 8, 2, 128
+    q, kp, vp, table, lens = _paged_case(77 + page, B, Hq, Hkv, d, page, 2100,
+                                         5000)
+    q = (q.float() * gain).to(torch.bfloat16)
+    out, st = paged_attention(q.cuda(), kp.cuda(), vp.cuda(), table.cuda(),
+                              lens.cuda(), 5000, normalizer=normalizer)
+    torch.cuda.synchronize()
+    assert nattn_get_device_status() == 0
+    res = oracle.paged_decode(q, kp, vp, table, lens, page, d ** -0.5,
+                              normalizer)
+    for b in range(B):
+        check_out(out[b].float().cpu().numpy(), res[b][0], f"seq {b}")
+        check_stat(st[b].cpu().numpy(), res[b][1], f"seq {b}")
+
+
 def test_paged_decode_bad_block_table_reports_bounds():
     """An out-of-range page id is caught on the device: the status word says
     NATTN_EBOUNDS and nothing faults."""
