@@ -97,6 +97,35 @@ __device__ __forceinline__ float fast_tanh(float x) {
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// tanh on the FMA pipe for |x| <= 1: x * q(x^2) with q of degree 4, fitted
+// for the smallest maximum absolute error on [-1, 1] by Lawson's algorithm
+// (csrc/tanh_poly.py computes the coefficients: error below 3e-6 in float32,
+// under the hardware tanh.approx's own on that interval).  Callers check the
+// range; outside it the polynomial is not tanh.
+struct TanhPoly {
+  float c[5];
+};
+// The coefficients scaled by `out`, so that the result is out * tanh(x).
+__device__ __forceinline__ void tanh_odd_coeffs(float out, TanhPoly& p) {
+  p.c[0] = 0.999968469f * out;
+  p.c[1] = -0.332658231f * out;
+  p.c[2] = 0.129220665f * out;
+  p.c[3] = -0.043299865f * out;
+  p.c[4] = 0.00836588722f * out;
+}
+// out * tanh(a * s) for two scores at once (packed f32x2 arithmetic).
+__device__ __forceinline__ void tanh_odd_poly2(float s0, float s1, float a, const TanhPoly& p,
+                                               float& z0, float& z1) {
+  float x0, x1, t0, t1, q0, q1;
+  ffma2(x0, x1, s0, s1, a, a, 0.f, 0.f);
+  ffma2(t0, t1, x0, x1, x0, x1, 0.f, 0.f);
+  ffma2(q0, q1, p.c[4], p.c[4], t0, t1, p.c[3], p.c[3]);
+  ffma2(q0, q1, q0, q1, t0, t1, p.c[2], p.c[2]);
+  ffma2(q0, q1, q0, q1, t0, t1, p.c[1], p.c[1]);
+  ffma2(q0, q1, q0, q1, t0, t1, p.c[0], p.c[0]);
+  ffma2(z0, z1, q0, q1, x0, x1, 0.f, 0.f);
+}
+
 // Three-input maximum (sm_100 `max.f32` with three sources).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float y;

@@ -182,7 +182,7 @@ __device__ __forceinline__ bool prefill_pair_normalizer(
     tmem_ld_wait();
     if (!fast) {
 #pragma unroll
-      for (int k = 0; k < BN; ++k) r[k] = __float_as_uint(tc_z(__uint_as_float(r[k]), A));
+      for (int c = 0; c < BN / 64; ++c) tc_z64(&r[c * 64], A);
     }
     if (edge) {
 #pragma unroll

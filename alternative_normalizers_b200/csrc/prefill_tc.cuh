@@ -210,6 +210,38 @@ __device__ __forceinline__ float tc_z(float s, const TcArgs& A) {
   return s * A.zscale;
 }
 
+// The same transform for 64 raw dot products held as bits.  With a soft-cap,
+// z = capscale * tanh(a s), a = scale / cap: when |a s| <= 1 for every score
+// of the warp (scores within the cap, the usual case) tanh comes from the odd
+// polynomial of tanh_odd_poly on the FMA pipe in packed pairs, leaving the
+// MUFU pipe to the exponentials; otherwise from tanh.approx.
+__device__ __forceinline__ void tc_z64(uint32_t* r, const TcArgs& A) {
+  if (A.P.softcap > 0.f) {
+    const float a = A.P.scale / A.P.softcap;
+    float amax = 0.f;
+#pragma unroll
+    for (int k = 0; k < 64; ++k) amax = fmaxf(amax, fabsf(__uint_as_float(r[k])));
+    if (__all_sync(0xffffffffu, amax * fabsf(a) <= 1.f)) {
+      TanhPoly c;
+      tanh_odd_coeffs(A.capscale, c);
+#pragma unroll
+      for (int k = 0; k < 64; k += 2) {
+        float z0, z1;
+        tanh_odd_poly2(__uint_as_float(r[k]), __uint_as_float(r[k + 1]), a, c, z0, z1);
+        r[k] = __float_as_uint(z0);
+        r[k + 1] = __float_as_uint(z1);
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 64; ++k)
+        r[k] = __float_as_uint(A.capscale * fast_tanh(__uint_as_float(r[k]) * a));
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 64; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * A.zscale);
+  }
+}
+
 // Exact threshold of N values held in registers (shifted threshold units;
 // -inf for no key) by tau_step from t0: every iterate is a lower bound of
 // the threshold.  Returns it in shifted units.
@@ -543,10 +575,7 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
       tmem_ld32(saddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
       tmem_ld32(saddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
       tmem_ld_wait();
-      if (!fast) {
-#pragma unroll
-        for (int k = 0; k < 64; ++k) r[k] = __float_as_uint(tc_z(__uint_as_float(r[k]), A));
-      }
+      if (!fast) tc_z64(r, A);
       if (edge) {
 #pragma unroll
         for (int k = 0; k < 64; ++k)

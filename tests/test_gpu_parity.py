@@ -91,6 +91,11 @@ TC_CASES = [
     (1, 2, 1, 200, 333, 128, True, 0, 0.0),      # Tq != Tk, bottom-right
     (1, 2, 2, 300, 100, 128, True, 0, 0.0),      # Tq > Tk: masked rows
     (1, 2, 1, 384, 384, 256, True, 0, 50.0),     # Gemma-like soft-cap
+    # cap 4: most 64-score chunks lie within the cap (polynomial tanh), a
+    # few hold a score past it (hardware tanh) in the same launch
+    (1, 2, 1, 384, 384, 256, True, 0, 4.0),
+    (1, 4, 2, 320, 320, 128, True, 0, 4.0),
+    (1, 4, 2, 320, 320, 128, True, 0, 50.0),     # soft-cap on the pair kernel
     (1, 2, 1, 600, 600, 128, True, 256, 0.0),    # sliding window
     (1, 2, 1, 300, 300, 128, True, 1000, 1.0),   # window >= T, heavy cap
     (1, 2, 1, 130, 130, 128, False, 50, 0.0),    # two-sided window
