@@ -575,7 +575,16 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
       tmem_ld32(saddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
       tmem_ld32(saddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
       tmem_ld_wait();
-      if (!fast) tc_z64(r, A);
+      if (!fast) {
+        if constexpr (MODE == TC_TAU) {
+          // per score: the packed polynomial form spills under this mode's
+          // register split
+#pragma unroll
+          for (int k = 0; k < 64; ++k) r[k] = __float_as_uint(tc_z(__uint_as_float(r[k]), A));
+        } else {
+          tc_z64(r, A);
+        }
+      }
       if (edge) {
 #pragma unroll
         for (int k = 0; k < 64; ++k)
