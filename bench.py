@@ -37,6 +37,12 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
                   "bf16_tflops_sustained": 1400.0}
 
 
+def peak_label(key, extra=""):
+    """'of measured <key>' or 'of fallback <key>', by where the peaks came
+    from (MEASURED_PEAKS.json, else the pool's earlier measurement)."""
+    return f"of {load_peaks()[1]} {key}{extra}"
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -848,11 +854,11 @@ def detail(args, dev, flush):
             peaks = load_peaks()[0]
             if w.paged:
                 frac = {n: round(v / peaks["hbm_gbs"], 4) for n, v in vals.items()}
-                fkind = "of measured hbm_gbs (dense-equivalent bytes)"
+                fkind = peak_label("hbm_gbs", " (dense-equivalent bytes)")
             else:
                 frac = {n: round(v / peaks["bf16_tflops"], 4)
                         for n, v in vals.items()}
-                fkind = "of measured bf16_tflops (burst)"
+                fkind = peak_label("bf16_tflops", " (burst)")
             res[name] = {"unit": unit, "value": vals,
                          "ms": {n: round(t, 4) for n, t in per.items()},
                          "roofline_frac": frac, "roofline_denominator": fkind}
@@ -887,7 +893,7 @@ def detail(args, dev, flush):
                 "value": vals, "ms": {n: round(t, 4) for n, t in per.items()},
                 "roofline_frac": {n: round(v / peaks["bf16_tflops"], 4)
                                   for n, v in vals.items()},
-                "roofline_denominator": "of measured bf16_tflops (burst)"}
+                "roofline_denominator": peak_label("bf16_tflops", " (burst)")}
             del r
             torch.cuda.empty_cache()
         except Exception as exc:
@@ -905,7 +911,7 @@ def detail(args, dev, flush):
             "unit": "useful TFLOP/s", "value": {"softmax+sinks": round(v, 1)},
             "ms": {"softmax+sinks": round(per["softmax"], 4)},
             "roofline_frac": {"softmax+sinks": round(v / peaks["bf16_tflops"], 4)},
-            "roofline_denominator": "of measured bf16_tflops (burst)"}
+            "roofline_denominator": peak_label("bf16_tflops", " (burst)")}
         del r, sinks
         torch.cuda.empty_cache()
     except Exception as exc:
@@ -932,7 +938,7 @@ def detail(args, dev, flush):
             "unit": "useful TFLOP/s (exact allowed pairs)", "value": vals,
             "ms": {n: round(t, 4) for n, t in per.items()},
             "roofline_frac": {n: round(v / peaks["bf16_tflops"], 4) for n, v in vals.items()},
-            "roofline_denominator": "of measured bf16_tflops (burst)"}
+            "roofline_denominator": peak_label("bf16_tflops", " (burst)")}
         del r, bm
         torch.cuda.empty_cache()
     except Exception as exc:
@@ -948,7 +954,7 @@ def detail(args, dev, flush):
                 "ms": {n: round(t, 4) for n, t in per.items()},
                 "roofline_frac": {n: round(v / peaks["bf16_tflops"], 4)
                                   for n, v in vals.items()},
-                "roofline_denominator": "of measured bf16_tflops (burst)"}
+                "roofline_denominator": peak_label("bf16_tflops", " (burst)")}
             del r
             torch.cuda.empty_cache()
         except Exception as exc:
