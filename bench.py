@@ -239,7 +239,10 @@ class Runner:
         return self.w.useful_flops()
 
 
-LAUNCHES = {"softmax": 1, "softmax1": 1, "sparsemax": 3, "entmax15": 3}
+# this library's kernels per call: the pair kernel for softmax / softmax1;
+# threshold pass, apply, wide and row-wise kernels for the sparse ones (the
+# last two exit at once when no row overflowed)
+LAUNCHES = {"softmax": 1, "softmax1": 1, "sparsemax": 4, "entmax15": 4}
 
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
 # capture of the current kernel (the profile summary named beside it).
@@ -248,6 +251,8 @@ NCU_TRAFFIC = {
     ("qwen3_8b_prefill", "softmax"): (
         131_183_872, "profiles/prefill_pair_qwen3_8b_softmax.md"),
 }
+# decode: split kernel and combine; sparse: score pass, threshold kernel,
+# apply pass and combine
 LAUNCHES_DECODE = {"softmax": 2, "softmax1": 2, "sparsemax": 4, "entmax15": 4}
 
 
