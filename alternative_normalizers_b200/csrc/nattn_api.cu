@@ -224,9 +224,10 @@ int validate(const nattn_args* a) {
   return NATTN_OK;
 }
 
-// Pages per decode split: 32 pages (2048 keys at 64-token pages) keeps every
-// CTA's loads several pages deep while the (sequence, kv head, split) grid of
-// the decode workload still fills two CTAs per SM many times over.
+// Pages per decode split: 32 pages (2048 keys at 64-token pages) give every
+// CTA a long run of pages to stream while the (sequence, kv head, split) grid
+// of the decode workload still fills the three to five CTAs each SM holds
+// many times over.
 constexpr int kDecodePagesPerSplit = 32;
 
 Plan make_plan(const nattn_args* a) {
