@@ -76,8 +76,22 @@ __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, 
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-// p_k = 2^(r_k * fa - m) for 64 scores held as raw bits; returns the bf16
+// p_k = 2^(r_k * fa - m) for N scores held as raw bits; returns the bf16
 // pairs packed for a TMEM store and adds the fp32 weights into s0 / s1.
+template <int N>
+__device__ __forceinline__ void exp2_packn(const uint32_t* r, float fa, float m, float& s0,
+                                           float& s1, uint32_t (&pk)[N / 2]) {
+#pragma unroll
+  for (int k = 0; k < N; k += 2) {
+    float x0, x1;
+    ffma2(x0, x1, __uint_as_float(r[k]), __uint_as_float(r[k + 1]), fa, fa, -m, -m);
+    const float p0 = fast_exp2(x0);
+    const float p1 = fast_exp2(x1);
+    fadd2(s0, s1, s0, s1, p0, p1);
+    pk[k >> 1] = pack_bf16(p0, p1);
+  }
+}
+// The same for 64 scores.
 // Pairs of scores share one f32x2 FFMA and one f32x2 add.
 __device__ __forceinline__ void exp2_pack64(const uint32_t* r, float fa, float m, float& s0,
                                             float& s1, uint32_t (&pk)[32]) {

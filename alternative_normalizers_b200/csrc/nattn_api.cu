@@ -431,8 +431,9 @@ int launch_tc(const nattn_args* a, const Problem& P, const Plan& pl, uint8_t* ws
         return check_launch();
       }
     }
-    // split each S row between two warps where TMEM holds two O halves
-    constexpr int NH = (2 * BN + 2 * D <= 512) ? 2 : 1;
+    // each S row split between two warps: two O halves where TMEM holds
+    // them, else one O the halves share (d = 256)
+    constexpr int NH = 2;
     using LY = TcLayout<D, D, BN, KST, VST, TC_ONLINE, NH>;
     auto k = prefill_tc_kernel<D, D, BN, KST, VST, TC_ONLINE, NH>;
     if (allow_smem(k, LY::ALLOC) != cudaSuccess) return NATTN_ECUDA;

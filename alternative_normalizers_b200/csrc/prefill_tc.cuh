@@ -146,6 +146,12 @@ __device__ __forceinline__ int value_row(const Problem& P, int b, int g, int j, 
 template <int D, int DV, int BN, int KST, int VST, int MODE, int NH = 1>
 struct TcLayout {
   static constexpr int NWN = 4 * NH;                 // normalizer warps
+  // Online, split rows where TMEM has no room for two O halves (d = 256:
+  // 2 x 64 + 2 x 256 > 512): the halves share one O and one running maximum
+  // (exchanged through shared memory every block), and each half writes its
+  // 32 keys' P for the same PV product.  Two normalizer warps per SM
+  // sub-partition instead of one.
+  static constexpr bool SHARED_O = MODE == TC_ONLINE && NH == 2 && 2 * BN + 2 * DV > 512;
   // The threshold pass with split rows holds a 64-score chunk, the bucket
   // maxima and the candidate state per thread: it runs three whole
   // warpgroups (two idle warps) so that setmaxnreg can move registers from
@@ -187,14 +193,18 @@ struct TcLayout {
   // epilogue (m, l) exchange between row halves: reuses the Q tile, which
   // every product has finished reading once the last PV has completed
   static constexpr int OFF_XCH = OFF_Q;
-  static constexpr int BYTES = OFF_MISC + 16;
+  // shared O: the halves' block maxima (by block parity) and, at the end,
+  // their denominators
+  static constexpr int OFF_XM = OFF_MISC + 16;
+  static constexpr int BYTES = OFF_XM + (SHARED_O ? 2 * 2 * TC_BM * 4 : 0);
   static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
   // TMEM columns: the S ring (NSB buffers of BN columns), then O (online)
   // or Q (threshold pass: bf16 pairs, D / 2 columns)
   static constexpr int TM_S = 0;  // S buffer s at column s * BN
   static constexpr int TM_O = 2 * BN;
   static constexpr int TM_Q = NSB * BN;
-  static constexpr int TM_COLS_USED = (MODE == TC_TAU) ? NSB * BN + D / 2 : 2 * BN + NH * DV;
+  static constexpr int TM_COLS_USED =
+      (MODE == TC_TAU) ? NSB * BN + D / 2 : 2 * BN + (SHARED_O ? DV : NH * DV);
   static constexpr int TM_COLS = TM_COLS_USED <= 32    ? 32
                                  : TM_COLS_USED <= 64  ? 64
                                  : TM_COLS_USED <= 128 ? 128
@@ -215,17 +225,18 @@ __device__ __forceinline__ float tc_z(float s, const TcArgs& A) {
 // of the warp (scores within the cap, the usual case) tanh comes from the odd
 // polynomial of tanh_odd_poly on the FMA pipe in packed pairs, leaving the
 // MUFU pipe to the exponentials; otherwise from tanh.approx.
-__device__ __forceinline__ void tc_z64(uint32_t* r, const TcArgs& A) {
+template <int N>
+__device__ __forceinline__ void tc_zn(uint32_t* r, const TcArgs& A) {
   if (A.P.softcap > 0.f) {
     const float a = A.P.scale / A.P.softcap;
     float amax = 0.f;
 #pragma unroll
-    for (int k = 0; k < 64; ++k) amax = fmaxf(amax, fabsf(__uint_as_float(r[k])));
+    for (int k = 0; k < N; ++k) amax = fmaxf(amax, fabsf(__uint_as_float(r[k])));
     if (__all_sync(0xffffffffu, amax * fabsf(a) <= 1.f)) {
       TanhPoly c;
       tanh_odd_coeffs(A.capscale, c);
 #pragma unroll
-      for (int k = 0; k < 64; k += 2) {
+      for (int k = 0; k < N; k += 2) {
         float z0, z1;
         tanh_odd_poly2(__uint_as_float(r[k]), __uint_as_float(r[k + 1]), a, c, z0, z1);
         r[k] = __float_as_uint(z0);
@@ -233,13 +244,28 @@ __device__ __forceinline__ void tc_z64(uint32_t* r, const TcArgs& A) {
       }
     } else {
 #pragma unroll
-      for (int k = 0; k < 64; ++k)
+      for (int k = 0; k < N; ++k)
         r[k] = __float_as_uint(A.capscale * fast_tanh(__uint_as_float(r[k]) * a));
     }
   } else {
 #pragma unroll
-    for (int k = 0; k < 64; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * A.zscale);
+    for (int k = 0; k < N; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * A.zscale);
   }
+}
+__device__ __forceinline__ void tc_z64(uint32_t* r, const TcArgs& A) { tc_zn<64>(r, A); }
+
+// Named barrier `id` over `nthreads` threads that also ANDs a flag across
+// them: every participant leaves with the same answer (used where a thread
+// that gave up a wait must not leave the others waiting at a barrier).
+__device__ __forceinline__ bool bar_and(int id, int nthreads, bool flag) {
+  uint32_t res;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(res)
+      : "r"(flag ? 1u : 0u), "r"(id), "r"(nthreads)
+      : "memory");
+  return res != 0;
 }
 
 // Exact threshold of N values held in registers (shifted threshold units;
@@ -443,8 +469,14 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
                 // operand, LBO = box stride, SBO = 8 key rows.
                 const uint64_t bd =
                     sdesc_sw128(vbase + (hh * NC + kk * 16) * 128, BN * 128, 1024);
-                umma_ts(tmem + LY::TM_O + hh * DV, pt + hh * NC + kk * 8, bd, IDESC_O,
-                        (jp > 0 || kk > 0) ? 1u : 0u);
+                if constexpr (LY::SHARED_O) {
+                  // both halves' keys into the one O
+                  umma_ts(tmem + LY::TM_O, pt + hh * NC + kk * 8, bd, IDESC_O,
+                          (jp > 0 || hh > 0 || kk > 0) ? 1u : 0u);
+                } else {
+                  umma_ts(tmem + LY::TM_O + hh * DV, pt + hh * NC + kk * 8, bd, IDESC_O,
+                          (jp > 0 || kk > 0) ? 1u : 0u);
+                }
               }
             }
             umma_commit(bar_vempty(vs));
@@ -495,6 +527,11 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
       const float sink2 = (half == 0) ? sink_logit(P, h) * 1.4426950408889634f : -INFINITY;
       m_run = sink2;
       l_run = (sink2 == -INFINITY) ? 0.f : 1.f;
+      if constexpr (LY::SHARED_O) {
+        // one running maximum for the row: both halves start from the sink,
+        // whose unit weight half 0 alone counts
+        m_run = sink_logit(P, h) * 1.4426950408889634f;
+      }
     } else {
       m_run = -INFINITY;
     }
@@ -553,7 +590,7 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
       thr = to_thr(lb);
     };
 
-    static_assert(NC == 64, "each normalizer thread owns 64 columns of a block");
+    static_assert(NC == 64 || LY::SHARED_O, "each normalizer thread owns 64 columns of a block");
     // Wait for S(j) and load this thread's 64 scores of key block kbc: z
     // (threshold / log2 units) unless the fast path keeps raw scores; masked
     // entries become -inf.  False when the wait was given up.
@@ -600,7 +637,86 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
     };
     const int kfirst = next_kept<BN>(P, b, h, h, qt, kb0, kend);
 
-    if constexpr (MODE == TC_ONLINE) {
+    if constexpr (MODE == TC_ONLINE && LY::SHARED_O) {
+      // Shared O: each half takes 32 of the block's 64 keys; the halves
+      // exchange their block maxima (by block parity) so that both move the
+      // one running maximum the same way, and each rescales half of O's
+      // columns.  Every barrier here also ANDs the warps' progress, so that
+      // all eight warps leave the loop together when a wait gives up.
+      float* xm = reinterpret_cast<float*>(smem + LY::OFF_XM);
+      bool ok_all = true;  // this warp's waits so far
+      int kbc = kfirst;
+      for (int j = 0; j < nblk; ++j, kbc = next_kept<BN>(P, b, h, h, qt, kbc + 1, kend)) {
+        const int sb = j % NSB;
+        const bool got =
+            __all_sync(0xffffffffu, mbar_wait_spin(bar_sfull(sb), (j / NSB) & 1, abort_flag));
+        uint32_t r[32];
+        float mx = -INFINITY;
+        const uint32_t saddr = lane_base + LY::TM_S + sb * BN + cbase;
+        if (got) {
+          tc_fence_after();
+          const int jb = kbc * BN + cbase;  // first key of this thread's columns
+          const bool edge = !(rr.lo <= jb && rr.hi >= jb + NC - 1);
+          int klb = rr.lo - jb;
+          unsigned span = (unsigned)(rr.hi - rr.lo);
+          if (rr.hi < rr.lo) {
+            klb = NC;
+            span = 0;
+          }
+          tmem_ld32(saddr, r);
+          tmem_ld_wait();
+          if (!fast) tc_zn<32>(r, A);
+          if (edge) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if ((unsigned)(k - klb) > span) r[k] = __float_as_uint(-INFINITY);
+          }
+          mx = max32_bits(r);
+          if (fast) mx *= zs;
+          xm[((j & 1) * 2 + half) * TC_BM + row] = mx;
+        }
+        if (!bar_and(2, NWN * 32, got && ok_all)) {
+          alive = false;
+          break;
+        }
+        mx = fmaxf(mx, xm[((j & 1) * 2 + (half ^ 1)) * TC_BM + row]);
+        const float mnew = fmaxf(m_run, mx);
+        const bool resc = mnew > m_run + 8.f;
+        const float m_use = resc ? mnew : m_run;
+        const float alpha = resc ? fast_exp2(m_run - mnew) : 1.f;
+        const float msafe = (m_use == -INFINITY) ? 0.f : m_use;
+        const float fa = fast ? zs : 1.f;  // p = exp2(x * fa - msafe)
+        float s0 = 0.f, s1 = 0.f;
+        uint32_t pk[16];  // 32 scores -> 16 packed columns at the start of this half's own
+        exp2_packn<32>(&r[0], fa, msafe, s0, s1, pk);
+        tmem_st16(saddr, pk);
+        tmem_st_wait();
+        l_run = l_run * alpha + (s0 + s1);
+        // rescale when the maximum moved, after PV(j-1) has completed; each
+        // half takes half of O's columns (both have the same alpha)
+        if (__any_sync(0xffffffffu, resc) && j > 0) {
+          if (__all_sync(0xffffffffu, mbar_wait_spin(bar_pv, (j - 1) & 1, abort_flag))) {
+            tc_fence_after();
+            const uint32_t oaddr = lane_base + LY::TM_O + half * (DV / 2);
+#pragma unroll 1
+            for (int c = 0; c < DV / 64; ++c) {
+              uint32_t o[32];
+              tmem_ld32(oaddr + c * 32, o);
+              tmem_ld_wait();
+#pragma unroll
+              for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+              tmem_st32(oaddr + c * 32, o);
+            }
+            tmem_st_wait();
+          } else {
+            ok_all = false;  // the next block's barrier takes every warp out
+          }
+        }
+        m_run = m_use;
+        release(j);
+      }
+      if (!ok_all) alive = false;
+    } else if constexpr (MODE == TC_ONLINE) {
       int kbc = kfirst;  // key block of step j
       for (int j = 0; j < nblk; ++j, kbc = next_kept<BN>(P, b, h, h, qt, kbc + 1, kend)) {
         uint32_t r[64];
@@ -870,9 +986,12 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
 #pragma unroll 1
       for (int c = 0; c < OC / 32; ++c) {
         uint32_t r[32], r1[32];
+        // (shared O: this half's columns of the one O, already both halves'
+        // sum)
+        constexpr bool TWO_O = NH > 1 && !LY::SHARED_O;
         if (have_o) {
           tmem_ld32(oaddr + c * 32, r);
-          if constexpr (NH > 1) tmem_ld32(oaddr + DV + c * 32, r1);
+          if constexpr (TWO_O) tmem_ld32(oaddr + DV + c * 32, r1);
           tmem_ld_wait();
         } else {
 #pragma unroll
@@ -882,7 +1001,7 @@ __global__ void __launch_bounds__((TcLayout<D, DV, BN, KST, VST, MODE, NH>::THRE
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
           o[k] = __uint_as_float(r[k]) * ca;
-          if constexpr (NH > 1) o[k] = fmaf(__uint_as_float(r1[k]), cb, o[k]);
+          if constexpr (TWO_O) o[k] = fmaf(__uint_as_float(r1[k]), cb, o[k]);
         }
         if (row_ok) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
