@@ -335,6 +335,16 @@ def e2e_measure(r, steps, dev):
     return ms, h2d, d2h * nn
 
 
+def e2e_chunks(B, Hkv):
+    """(batch entry, first KV head, end KV head) of each chunk of the
+    end-to-end loop: every batch entry, cut into two halves of its KV heads
+    (one piece when Hkv is odd).  A chunk's q rows (its KV heads' query
+    heads), k/v rows and out/row_stat rows are contiguous in the dense
+    layouts."""
+    gs = Hkv // 2 if Hkv % 2 == 0 else Hkv
+    return [(b, g0, g0 + gs) for b in range(B) for g0 in range(0, Hkv, gs)]
+
+
 def e2e_measure_dense(r, steps, dev):
     """The same metric through the C ABI with host buffers, as a serving loop
     would run it: every step copies its inputs from pinned host memory and
@@ -352,8 +362,7 @@ def e2e_measure_dense(r, steps, dev):
     import torch
     w = r.w
     grp = w.Hq // w.Hkv
-    gs = w.Hkv // 2 if w.Hkv % 2 == 0 else w.Hkv
-    chunks = [(b, g0, g0 + gs) for b in range(w.B) for g0 in range(0, w.Hkv, gs)]
+    chunks = e2e_chunks(w.B, w.Hkv)
     host = {k: r.host[k].pin_memory() for k in ("q", "k", "v")}
     din = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
     norms = list(w.normalizers)

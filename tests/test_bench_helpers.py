@@ -86,3 +86,19 @@ def test_sparse_decode_bytes_count_touched_v_pages(normalizer):
     assert got["total"] == kb + got["v_bytes"] + sb + got["qo_bytes"]
     # supports are small, so some V pages are never read
     assert 0 < touched < sum(-(-int(L) // ps) for L in x["seqlens"]) * w.Hkv
+
+
+@pytest.mark.parametrize("B,Hq,Hkv", [(2, 32, 8), (1, 16, 8), (3, 6, 3), (1, 4, 1)])
+def test_e2e_chunks_cover_heads_once_and_are_contiguous(B, Hq, Hkv):
+    """The end-to-end loop's chunks cover every (batch entry, KV head) exactly
+    once, and each chunk's slices of q [B, Hq, T, d] and k [B, Hkv, T, d] are
+    contiguous views (what a single copy per tensor and chunk relies on)."""
+    chunks = bench.e2e_chunks(B, Hkv)
+    seen = [(b, g) for b, g0, g1 in chunks for g in range(g0, g1)]
+    assert sorted(seen) == [(b, g) for b in range(B) for g in range(Hkv)]
+    grp = Hq // Hkv
+    q = torch.zeros(B, Hq, 5, 4)
+    k = torch.zeros(B, Hkv, 7, 4)
+    for b, g0, g1 in chunks:
+        assert q[b:b + 1, g0 * grp:g1 * grp].is_contiguous()
+        assert k[b:b + 1, g0:g1].is_contiguous()
