@@ -249,7 +249,7 @@ LAUNCHES = {"softmax": 1, "softmax1": 1, "sparsemax": 4, "entmax15": 4}
 # An entry is removed whenever the kernel changes after its capture.
 NCU_TRAFFIC = {
     ("qwen3_8b_prefill", "softmax"): (
-        131_183_872, "profiles/prefill_pair_qwen3_8b_softmax.md"),
+        131_220_224, "profiles/prefill_pair_qwen3_8b_softmax.md"),
 }
 # decode: split kernel and combine; sparse: score pass, threshold kernel,
 # apply pass and combine
